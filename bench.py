@@ -1,0 +1,479 @@
+#!/usr/bin/env python
+"""Benchmark of the SketchSSM decode hot path ("write full, read sketch") on B200.
+
+Workload: the Nemotron-Nano-9B-v2-shaped Mamba-2 layer (128 heads, K=128, V=80,
+8 basis groups, rank cap 49, mean rank 6, one dense-fallback head, W=16) at batch
+256 per GPU, synthetic seeded inputs.  One step = one window cycle of the whole hot
+path on every layer replica: W=16 sketch-decode launches, each followed on the last
+position by the flush (state update + sketch projection), i.e. B*W tokens per
+replica.  Layer replicas (default 8, about 1.8 GB each) rotate so that no decode
+finds its layer's data in the 126 MB L2 from the previous step.
+
+Printed JSON line (rank 0): value = tokens per second per SSM layer over all ranks,
+device time (CUDA events, max over ranks), plus the per-kernel roofline of the
+dominant kernel, the dense-read decode baseline, an end-to-end number through the
+C ABI with host-resident inputs, and the fp64 CPU oracle timed on the host cores.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decode tok/s per SSM layer at batch 256; HBM GB/s vs peak; speedup vs dense read"
+UNIT = "tok/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------- bytes
+
+def token_bytes(cfg) -> int:
+    """Bytes of one buffered token of one batch row: k (per q/k head), v, a, beta."""
+    da = cfg.K if cfg.kda else 1
+    return 4 * (cfg.Hqk * cfg.K + cfg.H * cfg.V + cfg.H * da + (cfg.H if cfg.has_beta else 0))
+
+
+def omega_bytes(cfg, rank) -> int:
+    Hg = cfg.H // cfg.G
+    rmax = [max([int(r) for r in rank[g * Hg:(g + 1) * Hg] if r > 0], default=0) for g in range(cfg.G)]
+    return 4 * cfg.K * sum(rmax)
+
+
+def decode_bytes(cfg, rank, pos: int) -> int:
+    """Algorithmic HBM bytes of one sketch-decode launch at buffer position pos:
+    per row the sketch rows of the sketch heads, the state of the dense heads, q, the
+    step's token (read, then appended), the pos earlier buffered tokens and y; plus
+    the basis rows once per launch."""
+    sk = [int(r) for r in rank if r > 0]
+    nd = sum(1 for r in rank if r <= 0)
+    row = (4 * cfg.V * sum(sk) + 4 * nd * cfg.K * cfg.V + 4 * cfg.Hqk * cfg.K
+           + (2 + pos) * token_bytes(cfg) + 4 * cfg.H * cfg.V)
+    return cfg.B * row + omega_bytes(cfg, rank)
+
+
+def dense_decode_bytes(cfg, pos: int) -> int:
+    """Same for the dense-read decode: the full state of every head instead of the sketch."""
+    row = (4 * cfg.H * cfg.K * cfg.V + 4 * cfg.Hqk * cfg.K + (2 + pos) * token_bytes(cfg)
+           + 4 * cfg.H * cfg.V)
+    return cfg.B * row
+
+
+def flush_bytes(cfg, rank, n: int) -> int:
+    """One flush of n buffered tokens: the state read and written once, the n tokens
+    read, the sketch written; plus the basis rows once per launch."""
+    sk = sum(int(r) for r in rank if r > 0)
+    row = 2 * 4 * cfg.H * cfg.K * cfg.V + n * token_bytes(cfg) + 4 * cfg.V * sk
+    return cfg.B * row + omega_bytes(cfg, rank)
+
+
+# ----------------------------------------------------------------------------- environment
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s)"
+
+
+def kernel_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's source
+    is unchanged since the counters were taken (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(ROOT, rec["source"])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["source_sha256"]:
+            return None
+        return rec
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = ["-i", str(self.device_index)]
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.out.read())) if len(r) >= 9]
+        self.out.close()
+        os.unlink(self.out.name)
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        sm, mx, reasons = [], [], set()
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_cycles(cfg, rank, omega, rows, min_s: float, max_cycles: int):
+    """Time whole window cycles (W decodes + the flush) of the fp64 oracle on `rows`."""
+    import oracle
+    S0 = synth.init_state(cfg, rows)
+    layer = oracle.OracleLayer(cfg.kind, H=cfg.H, Hqk=cfg.Hqk, K=cfg.K, V=cfg.V, W=cfg.W, G=cfg.G,
+                               rank=rank, omega=omega, S0=S0)
+    steps = [synth.step_inputs(cfg, t, rows) for t in range(cfg.W)]
+    layer.flush(0)
+    cycles, t0 = 0, time.perf_counter()
+    while True:
+        for p in range(cfg.W):
+            layer.decode(p, steps[p])
+        layer.flush(cfg.W)
+        cycles += 1
+        el = time.perf_counter() - t0
+        if el >= min_s or cycles >= max_cycles:
+            return cycles, el, oracle.num_threads()
+
+
+def cpu_baseline(cfg, rank, omega) -> dict:
+    rows = list(range(cfg.B))
+    cycles, el, threads = oracle_cycles(cfg, rank, omega, rows, min_s=10.0, max_cycles=64)
+    tok = cfg.B * cfg.W * cycles
+    return {"value": tok / el, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{cycles} window cycle(s) ({cycles * cfg.W} decode steps + {cycles} flushes) "
+                      f"of one layer at batch {cfg.B}, fp64, {el:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def replica_seed(rank_id: int, replica: int) -> int:
+    """Seed of one layer replica on one rank: every rank owns its own batch rows."""
+    return 1_000_003 * (rank_id + 1) + 7919 * replica
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity without a group)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_ours(args, cfg) -> None:
+    import torch
+    import torch.distributed as dist
+    import rank_state_read_b200 as rs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank_id = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    rank = synth.layer_rank_table(cfg)
+    omega = synth.basis(cfg)
+    L = args.replicas
+    layers, inputs = [], []
+    for l in range(L):
+        seed = replica_seed(rank_id, l)
+        S0 = synth.device_state(cfg, seed, dev)
+        layers.append(rs.SketchLayer(cfg.kind, batch=cfg.B, heads=cfg.H, qk_heads=cfg.Hqk,
+                                     key_dim=cfg.K, value_dim=cfg.V, window=cfg.W, groups=cfg.G,
+                                     rank_cap=cfg.cap, rank=rank.tolist(), omega=omega, S0=S0,
+                                     device=dev))
+        inputs.append([synth.device_step_inputs(cfg, seed + 1 + p, dev) for p in range(cfg.W)])
+        del S0
+    for lay in layers:
+        lay.flush(0)
+    torch.cuda.synchronize()
+
+    def cycle(dense=False, events=None):
+        for p in range(cfg.W):
+            for l, lay in enumerate(layers):
+                x = inputs[l][p]
+                if events is not None:
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                if dense:
+                    lay.dense_decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
+                else:
+                    lay.decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
+                if events is not None:
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e1.record(stream)
+                    events["decode"].append((p, e0, e1))
+                if p == cfg.W - 1 and not dense:
+                    if events is not None:
+                        e2 = torch.cuda.Event(enable_timing=True)
+                        e2.record(stream)
+                    lay.flush(cfg.W)
+                    if events is not None:
+                        e3 = torch.cuda.Event(enable_timing=True)
+                        e3.record(stream)
+                        events["flush"].append((cfg.W, e2, e3))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        cycle()
+    barrier()
+
+    # ---- timed region: K steps of the hot path
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ev = {"decode": [], "flush": []}
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        cycle(events=ev)
+    t_end.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_end)
+    dec = [(p, a.elapsed_time(b)) for p, a, b in ev["decode"]]
+    fl = [b_.elapsed_time(c_) for _, b_, c_ in ev["flush"]]
+    launches = len(ev["decode"]) + len(ev["flush"])
+
+    # ---- dense-read baseline decode (same positions, same replicas)
+    kd = max(1, min(args.steps, 10))
+    evd = {"decode": [], "flush": []}
+    barrier()
+    for _ in range(kd):
+        cycle(dense=True, events=evd)
+    barrier()
+    dd = [(p, a.elapsed_time(b)) for p, a, b in evd["decode"]]
+    for lay in layers:   # the dense-read cycles left W tokens buffered: apply them
+        lay.flush(cfg.W)
+
+    # ---- end to end through the C ABI: inputs from pinned host memory, y back to host
+    host_in = [{k: (None if v is None else v.cpu().pin_memory()) for k, v in inputs[0][p].items()}
+               for p in range(cfg.W)]
+    dev_in = {k: (None if v is None else torch.empty_like(v)) for k, v in inputs[0][0].items()}
+    host_y = [torch.empty(layers[0].y.shape, dtype=torch.float32).pin_memory() for _ in layers]
+    ke = max(1, min(args.steps, 5))
+    barrier()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    h2d = d2h = 0
+    for _ in range(ke):
+        for p in range(cfg.W):
+            for l, lay in enumerate(layers):
+                for k, v in host_in[p].items():
+                    if v is not None:
+                        dev_in[k].copy_(v, non_blocking=True)
+                        h2d += v.numel() * 4
+                y = lay.decode(p, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["a"], dev_in["beta"])
+                host_y[l].copy_(y, non_blocking=True)
+                d2h += y.numel() * 4
+                if p == cfg.W - 1:
+                    lay.flush(cfg.W)
+    e_end.record(stream)
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end)
+
+    # ---- max over ranks
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
+
+    tokens = cfg.B * cfg.W * L * args.steps * world
+    value = tokens / (ms / 1e3)
+    e2e_value = cfg.B * cfg.W * L * ke * world / (e2e_ms / 1e3)
+
+    peak, peak_src = hbm_peak()
+    dec_ms = sum(t for _, t in dec)
+    dec_bytes = sum(decode_bytes(cfg, rank, p) for p, _ in dec)
+    fl_ms = sum(fl)
+    fl_bytes = len(fl) * flush_bytes(cfg, rank, cfg.W)
+    dd_ms = sum(t for _, t in dd)
+    dd_bytes = sum(dense_decode_bytes(cfg, p) for p, _ in dd)
+    dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
+    fl_gbs = fl_bytes / (fl_ms / 1e3) / 1e9
+    dd_gbs = dd_bytes / (dd_ms / 1e3) / 1e9
+    mean_dec_us = 1e3 * dec_ms / len(dec)
+    mean_fl_us = 1e3 * fl_ms / len(fl)
+    mean_dd_us = 1e3 * dd_ms / len(dd)
+
+    def roof(kernel, achieved, nbytes_per_launch):
+        tr = kernel_traffic(kernel)
+        return {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": int(nbytes_per_launch),
+                "traffic": None if tr is None else tr["dram_bytes_per_launch_full_size"]}
+
+    share_dec = dec_ms / (dec_ms + fl_ms)
+    r_dec = roof("sketchssm_decode", dec_gbs, dec_bytes / len(dec))
+    r_fl = roof("sketchssm_flush", fl_gbs, fl_bytes / len(fl))
+    dominant, other = (r_dec, r_fl) if share_dec >= 0.5 else (r_fl, r_dec)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; shapes of the Nemotron Nano 9B v2 calibration card)",
+        "config": {"workload": cfg.name, "kind": cfg.kind, "batch_per_gpu": cfg.B, "heads": cfg.H,
+                   "K": cfg.K, "V": cfg.V, "groups": cfg.G, "qk_heads": cfg.Hqk, "window": cfg.W,
+                   "rank_cap": cfg.cap, "mean_rank": cfg.mean_rank, "dense_heads": int((rank < 0).sum()),
+                   "sketch_rows": int(rank[rank > 0].sum()), "layer_replicas": L,
+                   "step": f"{cfg.W} sketch decodes + 1 flush per replica",
+                   "l2": f"inputs larger than L2: {L} rotating layer replicas "
+                         f"({L * 1.8:.0f} GB), no L2 flush",
+                   "parallelism": f"batch sharded, {world} independent rank(s), no collective"},
+        "roofline": dominant,
+        "roofline_other": other,
+        "kernel_share": {"sketchssm_decode": round(share_dec, 4), "sketchssm_flush": round(1 - share_dec, 4)},
+        "decode_us": round(mean_dec_us, 2), "flush_us": round(mean_fl_us, 2),
+        "decode_only_tok_s": round(cfg.B * world / (mean_dec_us / 1e6), 1),
+        "dense_read": {"decode_us": round(mean_dd_us, 2), "hbm_gbs": round(dd_gbs, 1),
+                       "frac": round(dd_gbs / peak, 4),
+                       "decode_only_tok_s": round(cfg.B * world / (mean_dd_us / 1e6), 1)},
+        "speedup_vs_dense_read": round(mean_dd_us / mean_dec_us, 3),
+        "traffic_ratio_dense_over_sketch": round(dd_bytes / len(dd) / (dec_bytes / len(dec)), 3),
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d // ke,
+                "d2h_bytes_per_step": d2h // ke,
+                "note": "pinned host inputs copied in and y copied out around every decode call"},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank_id == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(cfg, rank, omega)
+    for lay in layers:
+        lay.close()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank_id == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, cfg) -> None:
+    """The reference arm of this pipeline is the fp64 CPU oracle as it stands: each
+    step is one window cycle of the same layer on a bounded sample of batch rows."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    rank = synth.layer_rank_table(cfg)
+    omega = synth.basis(cfg)
+    rows = list(range(args.ref_rows))
+    import oracle
+    S0 = synth.init_state(cfg, rows)
+    layer = oracle.OracleLayer(cfg.kind, H=cfg.H, Hqk=cfg.Hqk, K=cfg.K, V=cfg.V, W=cfg.W, G=cfg.G,
+                               rank=rank, omega=omega, S0=S0)
+    steps = [synth.step_inputs(cfg, t, rows) for t in range(cfg.W)]
+    layer.flush(0)
+
+    def cycle():
+        for p in range(cfg.W):
+            layer.decode(p, steps[p])
+        layer.flush(cfg.W)
+
+    for _ in range(args.warmup):
+        cycle()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cycle()
+    el = time.perf_counter() - t0
+    value = len(rows) * cfg.W * args.steps / el
+    threads = oracle.num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * el / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded; shapes of the Nemotron Nano 9B v2 calibration card)",
+            "config": {"workload": cfg.name, "kind": cfg.kind, "batch_per_gpu": cfg.B,
+                       "rows_per_step": len(rows), "step": f"{cfg.W} decodes + 1 flush"},
+            "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"{len(rows)} of {cfg.B} batch rows per step, "
+                                       f"{args.steps} window cycles"},
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", type=int, default=1, choices=(0, 1, 3, 4))
+    ap.add_argument("--replicas", type=int, default=8)
+    ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    cfg = synth.config(args.config)
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+/*
+ * sketchssm.h -- C ABI of the B200 (sm_100a) SketchSSM decode path.
+ *
+ * SketchSSM ("SketchSSM: Write to the Full State, Read from a Compact Sketch",
+ * paper abstract on the newx.sg and mlsanity pages) keeps the full fp32 recurrent
+ * state S (K x V per state head) up to date, but reads it only at state updates.
+ * Keys and values are buffered for a window of W tokens (ReplaySSM).  At each
+ * update (a "flush") the buffered tokens are applied to S and the new S is read
+ * once to form, for every sketch head, the r x V sketch Y = Omega_r S, Omega_r being
+ * the first r rows of the head group's fixed orthonormal basis.  Every decode step
+ * then forms the coefficients c = Omega_r q0 and returns
+ *     y = Y^T c + (exact replay of the buffered tokens),
+ * never touching S.  Heads allotted no rank ("dense fallback", sketchssm PyPI page,
+ * calibration stage "allocate") read S exactly.
+ *
+ * Recurrences (per state head, token i with key k_i, value v_i):
+ *     S <- M_i S + beta_i k_i v_i^T
+ *     Mamba-2 : M_i = a_i I,                        beta_i = 1   (a_i scalar)
+ *     GDN     : M_i = a_i (I - beta_i k_i k_i^T)                 (a_i scalar)
+ *     KDA     : M_i = diag(a_i) (I - beta_i k_i k_i^T)           (a_i in R^K)
+ * The output of a step is read after its own token is applied: y_t = S_t^T q_t.
+ *
+ * General conventions (every call):
+ *  - All tensors are fp32, C-contiguous, device memory owned by the caller, and
+ *    16-byte aligned (else SKETCHSSM_ERR_ALIGNMENT).  A pointer that is not device
+ *    accessible (plain host memory) is rejected with SKETCHSSM_ERR_INVALID_ARG.
+ *  - Layouts (B batch rows, H state heads, Hqk q/k heads, G basis groups, Rb basis
+ *    rows per group, W window, Rtot = sum of the sketch heads' ranks):
+ *        S     [B][H][K][V]         omega [G][Rb][K]       Y   [B][Rtot][V]
+ *        q, k  [B][Hqk][K]          v     [B][H][V]        y   [B][H][V]
+ *        a     [B][H]   (KDA [B][H][K])                    beta [B][H]
+ *        kbuf  [B][Hqk][W][K]       vbuf  [B][H][W][V]
+ *        abuf  [B][H][W] (KDA [B][H][W][K])                bbuf [B][H][W]
+ *    Head h belongs to basis group h / (H/G) and uses q/k head h / (H/Hqk).
+ *    Sketch head h owns rows off[h] .. off[h]+rank[h]-1 of Y (off = exclusive
+ *    prefix sum of the sketch ranks in head order; dense heads own no rows).
+ *  - beta and bbuf are ignored for Mamba-2 and may be NULL there.
+ *  - Every call is asynchronous and stream ordered (stream = a cudaStream_t, NULL
+ *    for the legacy default stream).  Arguments are checked on the host before any
+ *    launch; a call that returns an error launched nothing and wrote nothing.  A
+ *    failed launch returns SKETCHSSM_ERR_CUDA; sketchssm_last_error() then gives
+ *    the CUDA error text.  No call allocates or frees caller memory, and no kernel
+ *    waits on another CTA, so none can time out.
+ *  - Decode / flush protocol: pos counts the tokens buffered since the last flush.
+ *    sketchssm_decode(pos) appends the step's token at buffer slot pos and returns
+ *    y including it.  After the decode at pos = W-1 the caller runs
+ *    sketchssm_flush(n_tokens = W) and restarts at pos = 0.  sketchssm_flush with
+ *    n_tokens = 0 forms the sketch of an initial state.
+ *  - Supported shapes: K = 128, V a multiple of 16 in [16, 256], 1 <= W <= 32,
+ *    H divisible by G with H/G <= 32, Hqk dividing H and divisible by G,
+ *    1 <= rank_cap <= basis_rows <= K.  Others return SKETCHSSM_ERR_UNSUPPORTED.
+ *  - Calls on one plan from several host threads are safe; calls whose kernels
+ *    overlap on the GPU and write the same buffers race, as with any kernel.
+ */
+#ifndef SKETCHSSM_H
+#define SKETCHSSM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SKETCHSSM_OK = 0,
+    SKETCHSSM_ERR_INVALID_ARG = 1,  /* bad pointer, size, rank value or descriptor */
+    SKETCHSSM_ERR_ALIGNMENT = 2,    /* a tensor pointer is not 16-byte aligned */
+    SKETCHSSM_ERR_UNSUPPORTED = 3,  /* valid, but outside the shapes built for */
+    SKETCHSSM_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    SKETCHSSM_ERR_TIMEOUT = 5       /* reserved: no kernel of this library waits */
+} sketchssm_status;
+
+typedef enum {
+    SKETCHSSM_MAMBA2 = 0,  /* scalar decay per head ("Transformers are SSMs") */
+    SKETCHSSM_GDN = 1,     /* gated delta rule ("Gated Delta Networks") */
+    SKETCHSSM_KDA = 2      /* per-key-channel decay with the delta rule */
+} sketchssm_kind;
+
+/* rank-table value of a dense-fallback head (PyPI page, stage "allocate") */
+#define SKETCHSSM_DENSE (-1)
+
+/* Shape of one recurrent layer at a fixed batch. */
+typedef struct {
+    int32_t kind;        /* sketchssm_kind */
+    int32_t batch;       /* B >= 1 */
+    int32_t heads;       /* H: state heads */
+    int32_t qk_heads;    /* Hqk: heads carrying q and k (G for Mamba-2 groups, H per head) */
+    int32_t key_dim;     /* K (128 on the Nemotron Nano calibration card) */
+    int32_t value_dim;   /* V (80 on the card) */
+    int32_t window;      /* W (16 on the card) */
+    int32_t groups;      /* G: basis groups (8 on the card), contiguous runs of H/G heads */
+    int32_t basis_rows;  /* Rb: rows stored per group basis (79 on the card) */
+    int32_t rank_cap;    /* largest allowed rank (49 on the card) */
+} sketchssm_desc;
+
+/* Opaque plan: the layer's shape plus its device-side rank / offset / work tables. */
+typedef struct sketchssm_plan sketchssm_plan;
+
+/* A cudaStream_t, passed as a plain pointer. */
+typedef void *sketchssm_stream;
+
+/*
+ * Create a plan: checks desc, copies the per-head rank table (host, [H] int32,
+ * values SKETCHSSM_DENSE or 1..rank_cap) to the device and runs the layout kernel,
+ * which computes the packed sketch offsets off[H+1], the largest rank per group
+ * rmax[G] and the per-batch-row CTA work list (one item per dense head in head
+ * order, then one item per group holding a sketch head, in group order).  The plan
+ * owns those device tables (freed by sketchssm_plan_destroy).  Synchronises
+ * `stream` once, so that the host knows Rtot.  *out is set only on success.
+ * Source: the per-head "rank or a dense fallback" of the calibration stage
+ * "allocate" (sketchssm PyPI page) and the group-shared basis of stage "basis".
+ */
+sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t *rank_host,
+                                       sketchssm_stream stream, sketchssm_plan **out);
+
+/*
+ * Copy the plan's layout tables to host memory (synchronous).  Any output pointer
+ * may be NULL.  offsets_host gets H+1 values, rmax_host G values, work_host up to
+ * G+H entries (entry >= 0: group item g; entry < 0: dense item for head -entry-1)
+ * and *n_work their count.  *r_total gets Rtot, the number of sketch rows of Y.
+ */
+sketchssm_status sketchssm_plan_query(const sketchssm_plan *plan, int64_t *r_total,
+                                      int32_t *offsets_host, int32_t *rmax_host,
+                                      int32_t *work_host, int32_t *n_work);
+
+/* Free a plan and its device tables.  NULL is accepted.  Must not race with calls
+ * that use the plan; device work already queued keeps its own copy of nothing, so
+ * synchronise the streams that used the plan first. */
+sketchssm_status sketchssm_plan_destroy(sketchssm_plan *plan);
+
+/*
+ * Flush (write-full step; paper abstract: "preserves full-state updates" and "reads
+ * the full state once to precompute outputs for these basis vectors, storing them
+ * in a compact sketch").  For every (b, h) apply buffer slots 0..n_tokens-1 in
+ * order to S (in place), then write Y rows of every sketch head:
+ *     Y[b][off[h] + m][:] = sum_k omega[g(h)][m][k] S[b][h][k][:],  m < rank[h].
+ * n_tokens in [0, W]; with 0, S is left untouched and only Y is formed.
+ * Reads kbuf, vbuf, abuf, bbuf (slots < n_tokens), omega.  Writes S (if
+ * n_tokens > 0) and Y.  Y may be NULL only if the plan has no sketch head.
+ */
+sketchssm_status sketchssm_flush(const sketchssm_plan *plan, float *S, const float *omega,
+                                 const float *kbuf, const float *vbuf, const float *abuf,
+                                 const float *bbuf, int32_t n_tokens, float *Y,
+                                 sketchssm_stream stream);
+
+/*
+ * Sketch decode (read-sketch step; paper abstract: "combines the sketch vectors
+ * with query-dependent coefficients to reconstruct the output without a full-state
+ * read").  pos in [0, W): tokens buffered since the last flush.  Appends the step's
+ * token (k, v, a, beta) at buffer slot pos, then for every (b, h) with n = pos+1:
+ *   replay: walk the buffered tokens newest first with x = q,
+ *           y += beta_i (k_i . x) v_i,  x <- M_i^T x;      q0 = final x
+ *           (Mamba-2: y = sum_i w_i (k_i . q) v_i, w_i = prod_{j>i} a_j,
+ *            q0 = (prod_j a_j) q)
+ *   read:   sketch head: c = Omega_r q0, y += Y_h^T c;   dense head: y += S_h^T q0.
+ * Reads q, k, v, a, beta, the buffers' slots < pos, Y, omega and (dense heads
+ * only) S.  Writes y and buffer slot pos.  Y / omega may be NULL only if the plan
+ * has no sketch head; S may be NULL only if it has no dense head.
+ */
+sketchssm_status sketchssm_decode(const sketchssm_plan *plan, int32_t pos, const float *q,
+                                  const float *k, const float *v, const float *a,
+                                  const float *beta, float *kbuf, float *vbuf, float *abuf,
+                                  float *bbuf, const float *Y, const float *omega,
+                                  const float *S, float *y, sketchssm_stream stream);
+
+/*
+ * Dense-read decode: the ReplaySSM baseline the paper improves on ("each new query
+ * still requires a full-state read").  Same as sketchssm_decode, but every head
+ * reads S exactly (y += S_h^T q0) whatever its rank.  Reads S, never Y or omega.
+ */
+sketchssm_status sketchssm_dense_decode(const sketchssm_plan *plan, int32_t pos, const float *q,
+                                        const float *k, const float *v, const float *a,
+                                        const float *beta, float *kbuf, float *vbuf,
+                                        float *abuf, float *bbuf, const float *S, float *y,
+                                        sketchssm_stream stream);
+
+/* Static text of a status code. */
+const char *sketchssm_status_string(sketchssm_status status);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char *sketchssm_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKETCHSSM_H */

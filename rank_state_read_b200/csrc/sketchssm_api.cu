@@ -1,0 +1,411 @@
+// Host side of the C ABI declared in include/sketchssm.h: argument checks, the
+// plan (device rank / offset / work tables built by the layout kernel), and the
+// launches of the flush, sketch-decode and dense-read decode kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sketchssm_status fail(sketchssm_status s, const std::string &msg)
+{
+    g_last_error = msg;
+    return s;
+}
+
+sketchssm_status cuda_fail(cudaError_t e, const char *what)
+{
+    g_last_error = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+    return SKETCHSSM_ERR_CUDA;
+}
+
+// cuMemGetAddressRange through the runtime's driver entry point, so the library does
+// not link libcuda itself.
+typedef CUresult (*AddrRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+AddrRangeFn addr_range_fn()
+{
+    static AddrRangeFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return (AddrRangeFn) nullptr;
+        }
+        return (AddrRangeFn)p;
+    }();
+    return fn;
+}
+
+// A tensor argument must be 16-byte aligned device memory (of the current device,
+// or managed / mapped host memory) whose allocation holds `bytes` from `p` on.
+sketchssm_status check_tensor(const void *p, size_t bytes, const char *name, bool may_be_null)
+{
+    if (p == nullptr) {
+        if (may_be_null || bytes == 0) return SKETCHSSM_OK;
+        return fail(SKETCHSSM_ERR_INVALID_ARG, std::string(name) + " is NULL");
+    }
+    if (reinterpret_cast<uintptr_t>(p) % 16 != 0)
+        return fail(SKETCHSSM_ERR_ALIGNMENT, std::string(name) + " is not 16-byte aligned");
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(SKETCHSSM_ERR_INVALID_ARG, std::string(name) + " is not a CUDA pointer");
+    }
+    if (at.type == cudaMemoryTypeUnregistered ||
+        (at.type == cudaMemoryTypeHost && at.devicePointer == nullptr))
+        return fail(SKETCHSSM_ERR_INVALID_ARG, std::string(name) + " is not device-accessible memory");
+    if (at.type == cudaMemoryTypeDevice) {
+        int dev = -1;
+        cudaGetDevice(&dev);
+        if (at.device != dev)
+            return fail(SKETCHSSM_ERR_INVALID_ARG, std::string(name) + " lives on another device");
+        if (AddrRangeFn fn = addr_range_fn()) {
+            CUdeviceptr base = 0;
+            size_t size = 0;
+            if (fn(&base, &size, (CUdeviceptr)p) == CUDA_SUCCESS) {
+                const size_t avail = (size_t)(base + size - (CUdeviceptr)p);
+                if (bytes > avail)
+                    return fail(SKETCHSSM_ERR_INVALID_ARG,
+                                std::string(name) + " allocation is smaller than the tensor (" +
+                                    std::to_string(avail) + " < " + std::to_string(bytes) + " bytes)");
+            }
+        }
+    }
+    return SKETCHSSM_OK;
+}
+
+#define CHECK_T(ptr, bytes, name, nullable)                                    \
+    do {                                                                       \
+        sketchssm_status s_ = check_tensor((ptr), (bytes), (name), (nullable)); \
+        if (s_ != SKETCHSSM_OK) return s_;                                     \
+    } while (0)
+
+sketchssm_status check_desc(const sketchssm_desc *d)
+{
+    if (!d) return fail(SKETCHSSM_ERR_INVALID_ARG, "desc is NULL");
+    if (d->kind < SKETCHSSM_MAMBA2 || d->kind > SKETCHSSM_KDA)
+        return fail(SKETCHSSM_ERR_INVALID_ARG, "unknown kind");
+    if (d->batch < 1 || d->heads < 1 || d->qk_heads < 1 || d->groups < 1 || d->window < 1 ||
+        d->key_dim < 1 || d->value_dim < 1 || d->basis_rows < 1 || d->rank_cap < 1)
+        return fail(SKETCHSSM_ERR_INVALID_ARG, "every size in desc must be >= 1");
+    if (d->heads % d->groups != 0) return fail(SKETCHSSM_ERR_INVALID_ARG, "heads % groups != 0");
+    if (d->heads % d->qk_heads != 0) return fail(SKETCHSSM_ERR_INVALID_ARG, "heads % qk_heads != 0");
+    if (d->basis_rows > d->key_dim) return fail(SKETCHSSM_ERR_INVALID_ARG, "basis_rows > key_dim");
+    if (d->rank_cap > d->basis_rows) return fail(SKETCHSSM_ERR_INVALID_ARG, "rank_cap > basis_rows");
+    if (d->key_dim != sk::KDIM) return fail(SKETCHSSM_ERR_UNSUPPORTED, "key_dim must be 128");
+    if (d->value_dim % 16 != 0 || d->value_dim > sk::MAX_V)
+        return fail(SKETCHSSM_ERR_UNSUPPORTED, "value_dim must be a multiple of 16 in [16, 256]");
+    if (d->window > sk::MAX_W) return fail(SKETCHSSM_ERR_UNSUPPORTED, "window must be <= 32");
+    if (d->heads / d->groups > sk::MAX_HG) return fail(SKETCHSSM_ERR_UNSUPPORTED, "heads/groups must be <= 32");
+    if (d->qk_heads % d->groups != 0)
+        return fail(SKETCHSSM_ERR_UNSUPPORTED, "qk_heads must be a multiple of groups");
+    if (d->heads > (1 << 24)) return fail(SKETCHSSM_ERR_UNSUPPORTED, "too many heads");
+    return SKETCHSSM_OK;
+}
+
+sketchssm_status check_plan(const sketchssm_plan *p)
+{
+    if (!p) return fail(SKETCHSSM_ERR_INVALID_ARG, "plan is NULL");
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != p->device) return fail(SKETCHSSM_ERR_INVALID_ARG, "plan was created on another device");
+    return SKETCHSSM_OK;
+}
+
+size_t fbytes(long long a, long long b = 1, long long c = 1, long long d = 1)
+{
+    return (size_t)(a * b * c * d) * sizeof(float);
+}
+
+sk::DecodeArgs decode_args(const sketchssm_plan *p, int pos, const float *q, const float *k,
+                           const float *v, const float *a, const float *beta, float *kbuf,
+                           float *vbuf, float *abuf, float *bbuf, const float *Y,
+                           const float *omega, const float *S, float *y, int dense_all)
+{
+    const sketchssm_desc &d = p->d;
+    sk::DecodeArgs A;
+    A.kind = d.kind;
+    A.B = d.batch;
+    A.H = d.heads;
+    A.Hqk = d.qk_heads;
+    A.V = d.value_dim;
+    A.W = d.window;
+    A.G = d.groups;
+    A.Rb = d.basis_rows;
+    A.cap = d.rank_cap;
+    A.pos = pos;
+    A.Hg = p->Hg;
+    A.hpq = p->hpq;
+    A.rtot = p->rtot;
+    A.rank = p->d_rank;
+    A.off = p->d_off;
+    A.work = p->d_work;
+    A.n_work = p->n_work;
+    A.dense_all = dense_all;
+    sk::decode_threads(d.value_dim, &A.ns);
+    const int grp = p->max_group_rows + p->Hg * d.window;
+    const int den = sk::KDIM + d.window;
+    A.max_rows = grp > den ? grp : den;
+    A.q = q;
+    A.k = k;
+    A.v = v;
+    A.a = a;
+    A.beta = beta;
+    A.kbuf = kbuf;
+    A.vbuf = vbuf;
+    A.abuf = abuf;
+    A.bbuf = bbuf;
+    A.Y = Y;
+    A.omega = omega;
+    A.S = S;
+    A.y = y;
+    return A;
+}
+
+sketchssm_status check_decode_common(const sketchssm_plan *p, int pos, const float *q, const float *k,
+                                     const float *v, const float *a, const float *beta,
+                                     const float *kbuf, const float *vbuf, const float *abuf,
+                                     const float *bbuf, const float *y)
+{
+    const sketchssm_desc &d = p->d;
+    if (pos < 0 || pos >= d.window) return fail(SKETCHSSM_ERR_INVALID_ARG, "pos outside [0, window)");
+    const long long B = d.batch, H = d.heads, Q = d.qk_heads, K = d.key_dim, V = d.value_dim,
+                    W = d.window;
+    const long long da = d.kind == SKETCHSSM_KDA ? K : 1;
+    const bool mamba = d.kind == SKETCHSSM_MAMBA2;
+    CHECK_T(q, fbytes(B, Q, K), "q", false);
+    CHECK_T(k, fbytes(B, Q, K), "k", false);
+    CHECK_T(v, fbytes(B, H, V), "v", false);
+    CHECK_T(a, fbytes(B, H, da), "a", false);
+    CHECK_T(beta, mamba ? 0 : fbytes(B, H), "beta", mamba);
+    CHECK_T(kbuf, fbytes(B, Q, W, K), "kbuf", false);
+    CHECK_T(vbuf, fbytes(B, H, W, V), "vbuf", false);
+    CHECK_T(abuf, fbytes(B, H, W, da), "abuf", false);
+    CHECK_T(bbuf, mamba ? 0 : fbytes(B, H, W), "bbuf", mamba);
+    CHECK_T(y, fbytes(B, H, V), "y", false);
+    return SKETCHSSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sketchssm_status_string(sketchssm_status s)
+{
+    switch (s) {
+    case SKETCHSSM_OK: return "ok";
+    case SKETCHSSM_ERR_INVALID_ARG: return "invalid argument";
+    case SKETCHSSM_ERR_ALIGNMENT: return "misaligned tensor";
+    case SKETCHSSM_ERR_UNSUPPORTED: return "unsupported shape";
+    case SKETCHSSM_ERR_CUDA: return "CUDA error";
+    case SKETCHSSM_ERR_TIMEOUT: return "timeout";
+    }
+    return "unknown status";
+}
+
+const char *sketchssm_last_error(void) { return g_last_error.c_str(); }
+
+sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t *rank_host,
+                                       sketchssm_stream stream, sketchssm_plan **out)
+{
+    g_last_error.clear();
+    if (!out) return fail(SKETCHSSM_ERR_INVALID_ARG, "out is NULL");
+    sketchssm_status s = check_desc(desc);
+    if (s != SKETCHSSM_OK) return s;
+    if (!rank_host) return fail(SKETCHSSM_ERR_INVALID_ARG, "rank table is NULL");
+    const sketchssm_desc d = *desc;
+    const int H = d.heads, G = d.groups;
+    long long rtot = 0;
+    for (int h = 0; h < H; ++h) {
+        const int r = rank_host[h];
+        if (r == SKETCHSSM_DENSE) continue;
+        if (r < 1 || r > d.rank_cap)
+            return fail(SKETCHSSM_ERR_INVALID_ARG,
+                        "rank[" + std::to_string(h) + "] = " + std::to_string(r) +
+                            " is neither SKETCHSSM_DENSE nor in [1, rank_cap]");
+        rtot += r;
+    }
+    if (rtot > (1LL << 30)) return fail(SKETCHSSM_ERR_UNSUPPORTED, "too many sketch rows");
+
+    sketchssm_plan *p = new sketchssm_plan();
+    p->d = d;
+    p->Hg = H / G;
+    p->hpq = H / d.qk_heads;
+    cudaGetDevice(&p->device);
+    p->d_rank = p->d_off = p->d_rmax = p->d_work = p->d_counts = nullptr;
+    cudaStream_t st = (cudaStream_t)stream;
+    auto bail = [&](cudaError_t e, const char *what) {
+        sketchssm_plan_destroy(p);
+        return cuda_fail(e, what);
+    };
+    cudaError_t e;
+    if ((e = cudaMalloc(&p->d_rank, sizeof(int) * H)) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_off, sizeof(int) * (H + 1))) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_rmax, sizeof(int) * G)) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_work, sizeof(int) * (G + H))) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_counts, sizeof(int) * 4)) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMemcpyAsync(p->d_rank, rank_host, sizeof(int) * H, cudaMemcpyHostToDevice, st)) !=
+        cudaSuccess)
+        return bail(e, "cudaMemcpyAsync(rank)");
+    if ((e = sk::launch_layout(p->d_rank, H, G, d.rank_cap, p->d_off, p->d_rmax, p->d_work,
+                               p->d_counts, st)) != cudaSuccess)
+        return bail(e, "layout kernel launch");
+    int counts[4];
+    p->h_off.resize(H + 1);
+    p->h_rmax.resize(G);
+    p->h_work.resize(G + H);
+    if ((e = cudaMemcpyAsync(counts, p->d_counts, sizeof(counts), cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(p->h_off.data(), p->d_off, sizeof(int) * (H + 1), cudaMemcpyDeviceToHost, st)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(p->h_rmax.data(), p->d_rmax, sizeof(int) * G, cudaMemcpyDeviceToHost, st)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(p->h_work.data(), p->d_work, sizeof(int) * (G + H), cudaMemcpyDeviceToHost,
+                             st)) != cudaSuccess)
+        return bail(e, "cudaMemcpyAsync(layout)");
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return bail(e, "layout kernel");
+    if (counts[2] != 0) {
+        sketchssm_plan_destroy(p);
+        return fail(SKETCHSSM_ERR_INVALID_ARG, "layout kernel found an invalid rank");
+    }
+    p->n_work = counts[0];
+    p->n_dense = counts[1];
+    p->max_group_rows = counts[3];
+    p->rtot = p->h_off[H];
+    p->h_work.resize(p->n_work);
+    p->h_rank.assign(rank_host, rank_host + H);
+    if (p->rtot != rtot) {
+        sketchssm_plan_destroy(p);
+        return fail(SKETCHSSM_ERR_CUDA, "layout kernel disagrees with the host rank sum");
+    }
+    *out = p;
+    return SKETCHSSM_OK;
+}
+
+sketchssm_status sketchssm_plan_query(const sketchssm_plan *p, int64_t *r_total, int32_t *offsets_host,
+                                      int32_t *rmax_host, int32_t *work_host, int32_t *n_work)
+{
+    g_last_error.clear();
+    if (!p) return fail(SKETCHSSM_ERR_INVALID_ARG, "plan is NULL");
+    if (r_total) *r_total = p->rtot;
+    if (offsets_host) std::memcpy(offsets_host, p->h_off.data(), sizeof(int32_t) * p->h_off.size());
+    if (rmax_host) std::memcpy(rmax_host, p->h_rmax.data(), sizeof(int32_t) * p->h_rmax.size());
+    if (work_host) std::memcpy(work_host, p->h_work.data(), sizeof(int32_t) * p->h_work.size());
+    if (n_work) *n_work = p->n_work;
+    return SKETCHSSM_OK;
+}
+
+sketchssm_status sketchssm_plan_destroy(sketchssm_plan *p)
+{
+    if (!p) return SKETCHSSM_OK;
+    cudaFree(p->d_rank);
+    cudaFree(p->d_off);
+    cudaFree(p->d_rmax);
+    cudaFree(p->d_work);
+    cudaFree(p->d_counts);
+    delete p;
+    return SKETCHSSM_OK;
+}
+
+sketchssm_status sketchssm_flush(const sketchssm_plan *p, float *S, const float *omega, const float *kbuf,
+                                 const float *vbuf, const float *abuf, const float *bbuf, int32_t n_tokens,
+                                 float *Y, sketchssm_stream stream)
+{
+    g_last_error.clear();
+    sketchssm_status s = check_plan(p);
+    if (s != SKETCHSSM_OK) return s;
+    const sketchssm_desc &d = p->d;
+    if (n_tokens < 0 || n_tokens > d.window) return fail(SKETCHSSM_ERR_INVALID_ARG, "n_tokens outside [0, window]");
+    const long long B = d.batch, H = d.heads, Q = d.qk_heads, K = d.key_dim, V = d.value_dim, W = d.window;
+    const long long da = d.kind == SKETCHSSM_KDA ? K : 1;
+    const bool mamba = d.kind == SKETCHSSM_MAMBA2;
+    const bool any_sketch = p->rtot > 0;
+    const bool toks = n_tokens > 0;
+    CHECK_T(S, fbytes(B, H, K, V), "S", false);
+    CHECK_T(omega, any_sketch ? fbytes(d.groups, d.basis_rows, K) : 0, "omega", !any_sketch);
+    CHECK_T(Y, any_sketch ? fbytes(B, p->rtot, V) : 0, "Y", !any_sketch);
+    CHECK_T(kbuf, toks ? fbytes(B, Q, W, K) : 0, "kbuf", !toks);
+    CHECK_T(vbuf, toks ? fbytes(B, H, W, V) : 0, "vbuf", !toks);
+    CHECK_T(abuf, toks ? fbytes(B, H, W, da) : 0, "abuf", !toks);
+    CHECK_T(bbuf, (toks && !mamba) ? fbytes(B, H, W) : 0, "bbuf", !toks || mamba);
+    sk::FlushArgs A;
+    A.kind = d.kind;
+    A.B = d.batch;
+    A.H = d.heads;
+    A.Hqk = d.qk_heads;
+    A.V = d.value_dim;
+    A.W = d.window;
+    A.G = d.groups;
+    A.Rb = d.basis_rows;
+    A.cap = d.rank_cap;
+    A.n = n_tokens;
+    A.Hg = p->Hg;
+    A.hpq = p->hpq;
+    A.rtot = p->rtot;
+    A.rank = p->d_rank;
+    A.off = p->d_off;
+    A.S = S;
+    A.omega = omega;
+    A.kbuf = kbuf;
+    A.vbuf = vbuf;
+    A.abuf = abuf;
+    A.bbuf = bbuf;
+    A.Y = Y;
+    cudaError_t e = sk::launch_flush(A, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "flush kernel launch");
+    return SKETCHSSM_OK;
+}
+
+sketchssm_status sketchssm_decode(const sketchssm_plan *p, int32_t pos, const float *q, const float *k,
+                                  const float *v, const float *a, const float *beta, float *kbuf, float *vbuf,
+                                  float *abuf, float *bbuf, const float *Y, const float *omega, const float *S,
+                                  float *y, sketchssm_stream stream)
+{
+    g_last_error.clear();
+    sketchssm_status s = check_plan(p);
+    if (s != SKETCHSSM_OK) return s;
+    if ((s = check_decode_common(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, y)) != SKETCHSSM_OK)
+        return s;
+    const sketchssm_desc &d = p->d;
+    const bool any_sketch = p->rtot > 0, any_dense = p->n_dense > 0;
+    CHECK_T(Y, any_sketch ? fbytes(d.batch, p->rtot, d.value_dim) : 0, "Y", !any_sketch);
+    CHECK_T(omega, any_sketch ? fbytes(d.groups, d.basis_rows, d.key_dim) : 0, "omega", !any_sketch);
+    CHECK_T(S, any_dense ? fbytes(d.batch, d.heads, d.key_dim, d.value_dim) : 0, "S", !any_dense);
+    const sk::DecodeArgs A = decode_args(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, Y, omega, S, y, 0);
+    if (sk::decode_smem_bytes(A) > 200 * 1024)
+        return fail(SKETCHSSM_ERR_UNSUPPORTED, "decode item needs more than 200 KB of shared memory");
+    cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+    return SKETCHSSM_OK;
+}
+
+sketchssm_status sketchssm_dense_decode(const sketchssm_plan *p, int32_t pos, const float *q, const float *k,
+                                        const float *v, const float *a, const float *beta, float *kbuf,
+                                        float *vbuf, float *abuf, float *bbuf, const float *S, float *y,
+                                        sketchssm_stream stream)
+{
+    g_last_error.clear();
+    sketchssm_status s = check_plan(p);
+    if (s != SKETCHSSM_OK) return s;
+    if ((s = check_decode_common(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, y)) != SKETCHSSM_OK)
+        return s;
+    const sketchssm_desc &d = p->d;
+    CHECK_T(S, fbytes(d.batch, d.heads, d.key_dim, d.value_dim), "S", false);
+    const sk::DecodeArgs A = decode_args(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, nullptr, nullptr, S, y, 1);
+    if (sk::decode_smem_bytes(A) > 200 * 1024)
+        return fail(SKETCHSSM_ERR_UNSUPPORTED, "decode item needs more than 200 KB of shared memory");
+    cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "dense decode kernel launch");
+    return SKETCHSSM_OK;
+}
+
+}  // extern "C"

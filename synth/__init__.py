@@ -14,6 +14,8 @@ from .gen import (  # noqa: F401
     basis,
     basis_fp64,
     config,
+    device_state,
+    device_step_inputs,
     init_state,
     layer_rank_table,
     rank_table,

@@ -230,3 +230,42 @@ def step_inputs(cfg: Config, step: int, rows: Iterable[int], layer: int = 0) -> 
         if beta is not None:
             beta[j] = 1.0 / (1.0 + np.exp(-rng.standard_normal(cfg.H)))
     return {"q": q, "k": k, "v": v, "a": a, "beta": beta}
+
+
+# ----------------------------------------------------------------------------- device draws
+
+def device_state(cfg: Config, seed: int, device) -> "torch.Tensor":
+    """S0 with the distribution of ``init_state`` drawn by torch's generator on
+    ``device`` (other numbers than the numpy streams; for timing runs, where a
+    full-batch state of several GB would take minutes to draw on the host)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    S = torch.empty((cfg.B, cfg.H, cfg.K, cfg.V), dtype=torch.float32, device=device)
+    S.normal_(0.0, 0.1, generator=g)
+    return S
+
+
+def device_step_inputs(cfg: Config, seed: int, device) -> dict:
+    """One step's inputs with the distributions of ``step_inputs``, drawn on ``device``."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    f32 = dict(dtype=torch.float32, device=device)
+
+    def unit(shape):
+        z = torch.randn(shape, generator=g, **f32)
+        return z / z.norm(dim=-1, keepdim=True)
+
+    out = {"q": unit((cfg.B, cfg.Hqk, cfg.K)), "k": unit((cfg.B, cfg.Hqk, cfg.K)),
+           "v": torch.randn((cfg.B, cfg.H, cfg.V), generator=g, **f32)}
+    if cfg.kda:
+        lo = float(np.nextafter(np.float32(0.9), np.float32(1.0)))
+        hi = float(np.nextafter(np.float32(1.0), np.float32(0.0)))
+        out["a"] = (0.9 + 0.1 * torch.rand((cfg.B, cfg.H, cfg.K), generator=g, **f32)).clamp_(lo, hi)
+    else:
+        z = torch.randn((cfg.B, cfg.H), generator=g, **f32)
+        out["a"] = torch.exp(-torch.nn.functional.softplus(z) * 0.05)
+    out["beta"] = (torch.sigmoid(torch.randn((cfg.B, cfg.H), generator=g, **f32))
+                   if cfg.has_beta else None)
+    return out

@@ -1,0 +1,169 @@
+"""GPU (libsketchssm via its C ABI) against the fp64 oracle on the same seeded inputs.
+
+Bar: max |gpu - oracle| / max |oracle| <= 1e-4 for y at every decode step and for
+S and Y after every flush; the layout tables are compared bit for bit.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import parity_run
+
+pytestmark = pytest.mark.gpu
+DENSE = synth.DENSE
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from rank_state_read_b200 import build
+    build.build()
+
+
+def small(cid, **over):
+    return synth.config(cid).replace(**over)
+
+
+# ----------------------------------------------------------------------------- layout
+
+def layout_tables():
+    out = []
+    for cid in (0, 1, 3, 4):
+        cfg = synth.config(cid)
+        out.append((f"config{cid}", cfg, synth.layer_rank_table(cfg)))
+    for m in (4, 6, 10, 21):
+        cfg = synth.config(2, mean_rank=m, batch=64)
+        t = synth.stack_rank_tables(cfg)
+        for layer in (0, 13, 26):
+            out.append((f"stack-r{m}-l{layer}", cfg, t[layer]))
+    rng = np.random.default_rng(0)
+    cfg = synth.config(1)
+    for i in range(3):
+        r = rng.integers(1, cfg.cap + 1, cfg.H).astype(np.int32)
+        r[rng.random(cfg.H) < 0.3] = DENSE
+        out.append((f"random{i}", cfg, r))
+    out.append(("all-dense", cfg, np.full(cfg.H, DENSE, np.int32)))
+    out.append(("all-cap", cfg, np.full(cfg.H, cfg.cap, np.int32)))
+    return out
+
+
+@pytest.mark.parametrize("name,cfg,rank", layout_tables(), ids=[t[0] for t in layout_tables()])
+def test_layout_bit_exact(name, cfg, rank):
+    import rank_state_read_b200 as rs
+    plan = rs.Plan(cfg.kind, batch=1, heads=cfg.H, qk_heads=cfg.Hqk, key_dim=cfg.K, value_dim=cfg.V,
+                   window=cfg.W, groups=cfg.G, basis_rows=cfg.Rb, rank_cap=cfg.cap, rank=rank.tolist())
+    off, rmax, rtot = oracle.layout(rank, cfg.G)
+    assert plan.offsets == off.tolist()
+    assert plan.rmax == rmax.tolist()
+    assert plan.r_total == rtot
+    Hg = cfg.H // cfg.G
+    expect = [-h - 1 for h in range(cfg.H) if rank[h] == DENSE]
+    expect += [g for g in range(cfg.G) if (rank[g * Hg:(g + 1) * Hg] > 0).any()]
+    assert plan.work == expect
+    plan.close()
+
+
+# ----------------------------------------------------------------------------- small, every row
+
+def test_config0_full_trajectory():
+    """Tiny Mamba-2 layer, all 64 steps (4 flushes), every element."""
+    parity_run(synth.config(0), 64)
+
+
+def test_config0_dense_read_trajectory():
+    parity_run(synth.config(0), 40, dense=True)
+
+
+@pytest.mark.parametrize("cid,B", [(1, 3), (3, 3), (4, 2)])
+def test_layer_shapes_small_batch(cid, B):
+    """The pages' layer shapes at a small ragged batch: 2 flushes plus 7 buffered steps."""
+    parity_run(small(cid, B=B), 39)
+
+
+@pytest.mark.parametrize("cid,B", [(1, 3), (3, 2), (4, 2)])
+def test_dense_read_small_batch(cid, B):
+    parity_run(small(cid, B=B), 20, dense=True)
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+def test_all_heads_dense(kind):
+    cid = {"mamba2": 1, "gdn": 3, "kda": 4}[kind]
+    cfg = small(cid, B=2)
+    parity_run(cfg, 18, rank=np.full(cfg.H, DENSE, np.int32))
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+def test_all_heads_at_rank_cap(kind):
+    cid = {"mamba2": 1, "gdn": 3, "kda": 4}[kind]
+    cfg = small(cid, B=2)
+    parity_run(cfg, 18, rank=np.full(cfg.H, cfg.cap, np.int32))
+
+
+def test_rank_one_and_dense_mix():
+    cfg = small(1, B=2)
+    rank = np.ones(cfg.H, np.int32)
+    rank[::5] = DENSE
+    rank[:16] = DENSE            # group 0 has no sketch head at all
+    parity_run(cfg, 18, rank=rank)
+
+
+def test_partial_window_flushes():
+    """Flushes after 5, 16 and 3 more buffered tokens (n < W, then a fresh window)."""
+    parity_run(small(3, B=2), 30, flush_at=[5, 21, 24])
+
+
+def test_per_head_qk_mamba2():
+    """Mamba-2 with per-head q/k (Hqk = H): chains per head inside each group."""
+    parity_run(small(1, B=2, Hqk=128), 18)
+
+
+def test_shared_qk_gdn():
+    """GDN with q/k shared by the heads of a group (Hqk = G)."""
+    parity_run(small(3, B=2, Hqk=4), 18)
+
+
+@pytest.mark.parametrize("V,W,H,G", [(16, 5, 8, 2), (48, 7, 64, 2), (256, 32, 4, 1), (128, 1, 32, 1)])
+def test_other_shapes(V, W, H, G):
+    """Value dims, odd windows, 32 heads per group (the largest item), W = 1."""
+    cfg = small(3, B=2, V=V, W=W, H=H, G=G, Hqk=H, n_dense=1)
+    parity_run(cfg, 2 * W + 3)
+
+
+def test_single_row_batch():
+    parity_run(small(1, B=1), 17)
+
+
+# ----------------------------------------------------------------------------- full size, sampled rows
+
+FULL = [(1, 20), (3, 18), (4, 17)]
+
+
+@pytest.mark.parametrize("cid,T", FULL, ids=[f"config{c}" for c, _ in FULL])
+def test_full_size_sampled_rows(cid, T):
+    """The workloads at their full batch, in the bench's launch configuration; the
+    oracle computes a seeded sample of batch rows (rows are independent)."""
+    cfg = synth.config(cid)
+    rng = np.random.default_rng(cid)
+    rows = sorted({0, 1, cfg.B // 2, cfg.B - 1, *rng.integers(0, cfg.B, 3).tolist()})
+    parity_run(cfg, T, rows=rows)
+
+
+@pytest.mark.parametrize("cid", [1, 3])
+def test_full_size_dense_read_sampled_rows(cid):
+    cfg = synth.config(cid)
+    parity_run(cfg, 17, rows=[0, cfg.B // 3, cfg.B - 1], dense=True)
+
+
+@pytest.mark.parametrize("m", [4, 21])
+def test_stack_layer_sampled_rows(m):
+    """One layer of the 27-layer stack sweep (its own rank table: up to 22% dense)."""
+    cfg = synth.config(2, mean_rank=m, batch=256)
+    table = synth.stack_rank_tables(cfg)
+    layer = int(np.argmax((table == DENSE).sum(axis=1)))
+    one = cfg.replace(layers=1)
+    parity_run(one, 17, rank=table[layer], rows=[0, 100, 255])
