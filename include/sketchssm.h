@@ -39,8 +39,9 @@
  *    for the legacy default stream).  Arguments are checked on the host before any
  *    launch; a call that returns an error launched nothing and wrote nothing.  A
  *    failed launch returns SKETCHSSM_ERR_CUDA; sketchssm_last_error() then gives
- *    the CUDA error text.  No call allocates or frees caller memory, and no kernel
- *    waits on another CTA, so none can time out.
+ *    the CUDA error text.  No call allocates or frees caller memory.  No kernel
+ *    waits on another CTA; a decode CTA waits, with a bound, only for its own bulk
+ *    copies, and records a timeout that sketchssm_plan_check reports.
  *  - Decode / flush protocol: pos counts the tokens buffered since the last flush.
  *    sketchssm_decode(pos) appends the step's token at buffer slot pos and returns
  *    y including it.  After the decode at pos = W-1 the caller runs
@@ -67,7 +68,7 @@ typedef enum {
     SKETCHSSM_ERR_ALIGNMENT = 2,    /* a tensor pointer is not 16-byte aligned */
     SKETCHSSM_ERR_UNSUPPORTED = 3,  /* valid, but outside the shapes built for */
     SKETCHSSM_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
-    SKETCHSSM_ERR_TIMEOUT = 5       /* reserved: no kernel of this library waits */
+    SKETCHSSM_ERR_TIMEOUT = 5       /* a kernel gave up a bounded wait (sketchssm_plan_check) */
 } sketchssm_status;
 
 typedef enum {
@@ -103,10 +104,12 @@ typedef void *sketchssm_stream;
  * Create a plan: checks desc, copies the per-head rank table (host, [H] int32,
  * values SKETCHSSM_DENSE or 1..rank_cap) to the device and runs the layout kernel,
  * which computes the packed sketch offsets off[H+1], the largest rank per group
- * rmax[G] and the per-batch-row CTA work list (one item per dense head in head
- * order, then one item per group holding a sketch head, in group order).  The plan
- * owns those device tables (freed by sketchssm_plan_destroy).  Synchronises
- * `stream` once, so that the host knows Rtot.  *out is set only on success.
+ * rmax[G] and, for every number n = 1..W of replayed tokens, the CTA work list of
+ * one batch row of the decode launch: one item per dense head in head order, then
+ * per group its sketch heads packed greedily in head order into items whose rows
+ * (rank + n per head) fit one shared-memory stage.  The plan owns those device
+ * tables (freed by sketchssm_plan_destroy).  Synchronises `stream` once, so that
+ * the host knows Rtot and the item counts.  *out is set only on success.
  * Source: the per-head "rank or a dense fallback" of the calibration stage
  * "allocate" (sketchssm PyPI page) and the group-shared basis of stage "basis".
  */
@@ -114,14 +117,25 @@ sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t
                                        sketchssm_stream stream, sketchssm_plan **out);
 
 /*
- * Copy the plan's layout tables to host memory (synchronous).  Any output pointer
- * may be NULL.  offsets_host gets H+1 values, rmax_host G values, work_host up to
- * G+H entries (entry >= 0: group item g; entry < 0: dense item for head -entry-1)
- * and *n_work their count.  *r_total gets Rtot, the number of sketch rows of Y.
+ * Copy the plan's layout tables to host memory (reads host copies; no GPU work).
+ * Any output pointer may be NULL.  offsets_host gets H+1 values, rmax_host G
+ * values, *r_total Rtot (the number of sketch rows of Y), and work_host the work
+ * list for n_tokens (1..W) replayed tokens, at most G+H entries, *n_work their
+ * count.  Entry < 0: dense item for head -entry-1; entry >= 0: sketch item holding
+ * the sketch heads among heads entry/64 .. entry/64 + entry%64 - 1.
  */
 sketchssm_status sketchssm_plan_query(const sketchssm_plan *plan, int64_t *r_total,
-                                      int32_t *offsets_host, int32_t *rmax_host,
+                                      int32_t *offsets_host, int32_t *rmax_host, int32_t n_tokens,
                                       int32_t *work_host, int32_t *n_work);
+
+/*
+ * Synchronise `stream`, then report what the kernels recorded on the plan since the
+ * last check, and clear it: SKETCHSSM_ERR_TIMEOUT if a decode CTA gave up waiting
+ * (about a second) for its own bulk copies, in which case that call's y is
+ * incomplete; SKETCHSSM_OK otherwise.  No kernel waits on anything but its own
+ * copies, so a timeout means a fault of the copy engine, not a deadlock.
+ */
+sketchssm_status sketchssm_plan_check(const sketchssm_plan *plan, sketchssm_stream stream);
 
 /* Free a plan and its device tables.  NULL is accepted.  Must not race with calls
  * that use the plan; device work already queued keeps its own copy of nothing, so

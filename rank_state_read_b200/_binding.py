@@ -21,8 +21,8 @@ STATUS = {0: "SKETCHSSM_OK", 1: "SKETCHSSM_ERR_INVALID_ARG", 2: "SKETCHSSM_ERR_A
           3: "SKETCHSSM_ERR_UNSUPPORTED", 4: "SKETCHSSM_ERR_CUDA", 5: "SKETCHSSM_ERR_TIMEOUT"}
 
 # every symbol include/sketchssm.h declares
-EXPORTS = ("sketchssm_plan_create", "sketchssm_plan_query", "sketchssm_plan_destroy",
-           "sketchssm_flush", "sketchssm_decode", "sketchssm_dense_decode",
+EXPORTS = ("sketchssm_plan_create", "sketchssm_plan_query", "sketchssm_plan_check",
+           "sketchssm_plan_destroy", "sketchssm_flush", "sketchssm_decode", "sketchssm_dense_decode",
            "sketchssm_status_string", "sketchssm_last_error")
 
 
@@ -52,12 +52,13 @@ def load():
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
     lib.sketchssm_plan_create.argtypes = [ctypes.POINTER(Desc), P, P, ctypes.POINTER(P)]
-    lib.sketchssm_plan_query.argtypes = [P, ctypes.POINTER(I64), P, P, P, ctypes.POINTER(I32)]
+    lib.sketchssm_plan_query.argtypes = [P, ctypes.POINTER(I64), P, P, I32, P, ctypes.POINTER(I32)]
+    lib.sketchssm_plan_check.argtypes = [P, P]
     lib.sketchssm_plan_destroy.argtypes = [P]
     lib.sketchssm_flush.argtypes = [P, P, P, P, P, P, P, I32, P, P]
     lib.sketchssm_decode.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.sketchssm_dense_decode.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P]
-    for f in EXPORTS[:6]:
+    for f in EXPORTS[:7]:
         getattr(lib, f).restype = ctypes.c_int
     lib.sketchssm_status_string.argtypes = [ctypes.c_int]
     lib.sketchssm_status_string.restype = ctypes.c_char_p
@@ -115,18 +116,22 @@ class Plan:
         self.handle = handle
         self.rank = [int(r) for r in rank]
         rt = ctypes.c_int64()
-        nw = ctypes.c_int32()
         off = (ctypes.c_int32 * (heads + 1))()
         rmax = (ctypes.c_int32 * groups)()
-        work = (ctypes.c_int32 * (groups + heads))()
         _check(lib.sketchssm_plan_query(handle, ctypes.byref(rt), ctypes.cast(off, ctypes.c_void_p),
-                                        ctypes.cast(rmax, ctypes.c_void_p),
-                                        ctypes.cast(work, ctypes.c_void_p), ctypes.byref(nw)),
+                                        ctypes.cast(rmax, ctypes.c_void_p), 1, None, None),
                "sketchssm_plan_query")
         self.r_total = int(rt.value)
         self.offsets = list(off)
         self.rmax = list(rmax)
-        self.work = list(work)[: nw.value]
+        self.work = {}
+        for n in range(1, window + 1):
+            nw = ctypes.c_int32()
+            work = (ctypes.c_int32 * (groups + heads))()
+            _check(lib.sketchssm_plan_query(handle, None, None, None, n,
+                                            ctypes.cast(work, ctypes.c_void_p), ctypes.byref(nw)),
+                   "sketchssm_plan_query")
+            self.work[n] = list(work)[: nw.value]
 
     # shapes of the caller-owned tensors (include/sketchssm.h, "Layouts")
     @property
@@ -144,6 +149,10 @@ class Plan:
         for x in self.shapes[name]:
             n *= x
         return n
+
+    def check(self, stream=None) -> None:
+        """Synchronise and raise if a kernel recorded a timeout (sketchssm_plan_check)."""
+        _check(load().sketchssm_plan_check(self.handle, _stream(stream)), "sketchssm_plan_check")
 
     def close(self) -> None:
         if getattr(self, "handle", None) is not None and self.handle.value:

@@ -1,4 +1,4 @@
-// Sketch decode and dense-read decode (one launch per decode step).
+// Sketch decode and dense-read decode: two launches per decode step.
 //
 // Paper abstract (SketchSSM, newx.sg / mlsanity pages): a decode step "combines the
 // sketch vectors with query-dependent coefficients to reconstruct the output
@@ -7,379 +7,557 @@
 // stage "allocate") reads the full state instead; the dense-read baseline does that
 // for every head.
 //
-// One CTA per (work item, batch row).  A work item is either
-//   - a group item: all sketch heads of one basis group (they share Omega_g and,
-//     for Mamba-2 with group-shared B/C, the query and keys), or
-//   - a dense item: one head whose base rows are its K state rows.
-// Every head of an item contributes a list of rows, each a V-vector with a scalar
-// coefficient: its base rows (sketch rows of Y, or state rows of S) and its n
-// buffered value rows.  The output of the head is the weighted sum of its rows.
+// Every head's output is a weighted sum of rows of V floats: its base rows (the r
+// sketch rows of Y, or the K state rows of S for a dense head) and its n buffered
+// value rows.  The step splits into
 //
-// Phase A computes the coefficients into shared memory:
-//   Mamba-2: per q/k head s_i = k_i . q and u_m = Omega_g[m] . q (one warp per dot),
-//            per head the suffix products w_i = prod_{j>i} a_j and decay_prod;
-//            base coefficient decay_prod * u_m (sketch) or decay_prod * q_k (dense),
-//            replay coefficient w_i s_i.
-//   GDN/KDA: per head one warp walks the buffer newest first, x <- M_i^T x, with
-//            replay coefficient beta_i (k_i . x); then q0 = x and the base
-//            coefficients Omega_g[m] . q0 (sketch) or q0 itself (dense).
-// Phase B streams every row once with 16-byte loads.  The item's row list is cut
-// into `ns` contiguous chunks, one per slice of V/4 threads; each slice sums its
-// chunk per head into a shared partial, and the partials of a head are added in
-// slice order, so the result does not depend on scheduling.
-// The step's own token is read from the inputs and appended at buffer slot pos
-// (keys by the item that owns the first head of their q/k head).
+//  1. the query-side products, written to the plan's scratch:
+//     Mamba-2 (dots_kernel_mamba2), one CTA per (q/k head, up to 8 batch rows): the
+//       group's basis rows, the rows' queries and buffered keys are staged in shared
+//       memory in one round; s_i = k_i . q (one lane per key) and
+//       u_m = Omega_g[m] . q (register-blocked over the CTA's rows) are written per
+//       (batch row, q/k head).  The step's key is appended to buffer slot pos.
+//     GDN/KDA (coef_kernel_delta), one warp per (batch row, head): walk the buffer
+//       newest first, x <- M_i^T x, keys (and KDA decays) prefetched four steps
+//       ahead; the replay coefficients beta_i (k_i . x) and the base coefficients
+//       Omega_g[m] . q0 (sketch) or q0 = x (dense) are written per head.  The step's
+//       key, decay and beta are appended to buffer slot pos.
+//  2. combine_kernel, one CTA per (work item, batch row): the layout kernel packs
+//     the sketch heads of a basis group into items whose rows fit one shared-memory
+//     stage (a dense head is an item of its own).  Warp 0 issues bulk (TMA) copies of
+//     the item's block of Y (or the head's state), every buffered value row, the
+//     step's values and the products of step 1, all counted on one mbarrier (the
+//     item's record from the layout kernel is the only load on the path to the
+//     copies; it is launched as a programmatic dependent of step 1 and waits for it
+//     only before copying step 1's products).  After a bounded wait, thread (head,
+//     column chunk) sums its head's
+//     rows in row order (deterministic) and writes y.  For Mamba-2 the coefficients
+//     are formed on the fly: walking the buffer newest first with w = 1,
+//     row i gets w s_i and w <- w a_i, so that w ends as decay_prod; base row m then
+//     gets decay_prod u_m (sketch) or decay_prod q_m (dense).  The step's value (and
+//     Mamba-2's decay) is appended to buffer slot pos.
 #include "device_util.cuh"
 #include "internal.cuh"
+#include "ptx_util.cuh"
 
 namespace sk {
 namespace {
 
-constexpr int DECODE_THREADS_TARGET = 320;
-constexpr int DECODE_MAX_THREADS = 384;
-constexpr int UNROLL = 8;
+constexpr int COMBINE_TARGET_THREADS = 160;
+constexpr int STAGE_TARGET = 40 * 1024;  // bytes of rows of a typical sketch item
+constexpr int MAXC = 32;
+constexpr int COEF_THREADS = 128;
+
+__host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
+
+// ============================================================================ query-side products
+
+constexpr int CM_THREADS = 256;
+constexpr int CM_MAXROWS = 8;
+constexpr int OPAD = KDIM + 4;  // padded row: threads reading different rows hit different banks
+
+struct CmCarve {
+    size_t om, ks, qs, sd, ud, total;
+};
+
+__host__ __device__ inline size_t cm_take(size_t &o, size_t bytes)
+{
+    const size_t r = o;
+    o = (o + bytes + 127) & ~size_t(127);
+    return r;
+}
+
+__host__ __device__ inline CmCarve cm_carve(int cap, int W, int rows)
+{
+    CmCarve c;
+    size_t o = 0;
+    c.om = cm_take(o, sizeof(float) * (size_t)cap * OPAD);
+    c.ks = cm_take(o, sizeof(float) * (size_t)rows * W * OPAD);
+    c.qs = cm_take(o, sizeof(float) * (size_t)rows * KDIM);
+    c.sd = cm_take(o, sizeof(float) * (size_t)rows * W);
+    c.ud = cm_take(o, sizeof(float) * (size_t)rows * cap);
+    c.total = o;
+    return c;
+}
+
+// Mamba-2: one CTA per (q/k head, `rows` batch rows).  Output per (batch row, q/k
+// head): dots_row floats, s_0 .. s_{W-1} then u_0 .. u_{cap-1} (unused entries 0).
+__global__ void __launch_bounds__(CM_THREADS)
+dots_kernel_mamba2(const DecodeArgs A)
+{
+    extern __shared__ __align__(128) unsigned char cms[];
+    pdl_launch_dependents();  // the combine may start staging its rows now
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int W = A.W, pos = A.pos, n = pos + 1, hpq = A.hpq, cap = A.cap;
+    const int rows = A.cm_rows;
+    const int q = blockIdx.x, b0 = blockIdx.y * rows;
+    const int nb = min(rows, A.B - b0);
+    const int g = (q * hpq) / A.Hg;
+    const CmCarve cv = cm_carve(cap, W, rows);
+    float *om = reinterpret_cast<float *>(cms + cv.om);     // [cap][OPAD]
+    float *ks = reinterpret_cast<float *>(cms + cv.ks);     // [rows][W][OPAD] keys (slot pos: the step's)
+    float *qs = reinterpret_cast<float *>(cms + cv.qs);     // [rows][K]
+    float *s_dot = reinterpret_cast<float *>(cms + cv.sd);  // [rows][W]
+    float *u_dot = reinterpret_cast<float *>(cms + cv.ud);  // [rows][cap]
+
+    const int orows = A.dense_all ? 0 : cap;
+    const float *og = A.omega + (long long)g * A.Rb * KDIM;
+    for (int x = tid; x < orows * (KDIM / 4); x += CM_THREADS) {
+        const int j = x >> 5, c = x & 31;
+        cp_async16(om + j * OPAD + c * 4, og + (long long)j * KDIM + c * 4);
+    }
+    for (int x = tid; x < nb * (KDIM / 4); x += CM_THREADS) {
+        const int bl = x >> 5, c = x & 31;
+        cp_async16(qs + bl * KDIM + c * 4, A.q + ((long long)(b0 + bl) * A.Hqk + q) * KDIM + c * 4);
+    }
+    for (int x = tid; x < nb * n * (KDIM / 4); x += CM_THREADS) {
+        const int c = x & 31, r = x >> 5, bl = r / n, i = r - bl * n;
+        const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
+        cp_async16(ks + (bl * W + i) * OPAD + c * 4,
+                   (i == pos ? A.k + qrow * KDIM : A.kbuf + (qrow * W + i) * KDIM) + c * 4);
+    }
+    const int rq = A.dense_all ? 0 : __ldg(A.qk_rneed + q);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    if (warp < 4) {
+        // u[bl][j] = Omega_g[j] . q_bl: thread j, all batch rows at once
+        for (int j = tid; j < rq; j += 128) {
+            const float *orow = om + (size_t)j * OPAD;
+            float acc[CM_MAXROWS];
+#pragma unroll
+            for (int bl = 0; bl < CM_MAXROWS; ++bl) acc[bl] = 0.f;
+#pragma unroll 4
+            for (int c = 0; c < KDIM; c += 4) {
+                const float4 o = lds4(orow + c);
+#pragma unroll
+                for (int bl = 0; bl < CM_MAXROWS; ++bl) {
+                    if (bl < nb) {
+                        const float4 x = lds4(qs + bl * KDIM + c);
+                        acc[bl] = fmaf(o.x, x.x, fmaf(o.y, x.y, fmaf(o.z, x.z, fmaf(o.w, x.w, acc[bl]))));
+                    }
+                }
+            }
+#pragma unroll
+            for (int bl = 0; bl < CM_MAXROWS; ++bl)
+                if (bl < nb) u_dot[bl * cap + j] = acc[bl];
+        }
+    } else {
+        // s[bl][i] = k_i . q_bl: a half warp per batch row, lane i per key
+        const int half = (warp - 4) * 2 + (lane >> 4), i0 = lane & 15;
+        for (int bl = half; bl < nb; bl += 8) {
+            const float *qb = qs + bl * KDIM;
+            for (int i = i0; i < n; i += 16) {
+                const float *row = ks + (bl * W + i) * OPAD;
+                float4 acc = zero4();
+#pragma unroll 8
+                for (int c = 0; c < KDIM; c += 4) {
+                    const float4 o = lds4(row + c), x = lds4(qb + c);
+                    acc.x = fmaf(o.x, x.x, acc.x);
+                    acc.y = fmaf(o.y, x.y, acc.y);
+                    acc.z = fmaf(o.z, x.z, acc.z);
+                    acc.w = fmaf(o.w, x.w, acc.w);
+                }
+                s_dot[bl * W + i] = (acc.x + acc.y) + (acc.z + acc.w);
+            }
+        }
+    }
+    // the step's key goes to buffer slot pos (from the stage)
+    for (int x = tid; x < nb * (KDIM / 4); x += CM_THREADS) {
+        const int bl = x >> 5, c = x & 31;
+        const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
+        st4(A.kbuf + (qrow * W + pos) * KDIM + c * 4, lds4(ks + (bl * W + pos) * OPAD + c * 4));
+    }
+    __syncthreads();
+    const int dr = A.dots_row;
+    for (int x = tid; x < nb * dr; x += CM_THREADS) {
+        const int bl = x / dr, e = x - bl * dr;
+        float v = 0.f;
+        if (e < W) {
+            if (e < n) v = s_dot[bl * W + e];
+        } else if (e - W < rq) {
+            v = u_dot[bl * cap + (e - W)];
+        }
+        A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + e] = v;
+    }
+}
+
+// GDN / KDA: one warp per (head, batch row).
+template <int KIND>
+__global__ void __launch_bounds__(COEF_THREADS)
+coef_kernel_delta(const DecodeArgs A)
+{
+    pdl_launch_dependents();  // the combine may start staging its rows now
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int h = blockIdx.x * (COEF_THREADS / 32) + warp, b = blockIdx.y;
+    const int H = A.H, W = A.W, pos = A.pos, n = pos + 1, hpq = A.hpq;
+    if (h >= H) return;
+    const int qk = h / hpq, g = h / A.Hg;
+    const long long bh = (long long)b * H + h;
+    const long long qrow = (long long)b * A.Hqk + qk;
+    const int r = __ldg(A.rank + h);
+    const bool dense = A.dense_all || r <= 0;
+    const int rb = dense ? KDIM : r;
+    float *dst = A.scratch + (long long)b * A.coef_row +
+                 (A.dense_all ? (long long)h * A.coef_dense_block : __ldg(A.coff + h));
+
+    float bl = 0.f, al = 0.f;
+    if (lane < n) {
+        bl = (lane == pos) ? __ldg(A.beta + bh) : __ldg(A.bbuf + bh * W + lane);
+        if (KIND == SKETCHSSM_GDN) al = (lane == pos) ? __ldg(A.a + bh) : __ldg(A.abuf + bh * W + lane);
+    }
+    if (lane == pos) {
+        A.bbuf[bh * W + pos] = bl;
+        if (KIND == SKETCHSSM_GDN) A.abuf[bh * W + pos] = al;
+    }
+    const float *kcur = A.k + qrow * KDIM + lane * 4;
+    const float *kb = A.kbuf + qrow * W * KDIM + lane * 4;
+    const float *acur = A.a + bh * KDIM + lane * 4;      // KDA
+    const float *ab = A.abuf + bh * W * KDIM + lane * 4;  // KDA
+    auto kl = [&](int i) { return i == pos ? ldg4(kcur) : ldg4(kb + (long long)i * KDIM); };
+    auto al4 = [&](int i) { return i == pos ? ldg4(acur) : ldg4(ab + (long long)i * KDIM); };
+    const float4 z = zero4();
+    float4 k0 = kl(n - 1), k1 = n >= 2 ? kl(n - 2) : z, k2 = n >= 3 ? kl(n - 3) : z, k3 = n >= 4 ? kl(n - 4) : z;
+    float4 a0 = z, a1 = z, a2 = z, a3 = z;
+    if (KIND == SKETCHSSM_KDA) {
+        a0 = al4(n - 1);
+        if (n >= 2) a1 = al4(n - 2);
+        if (n >= 3) a2 = al4(n - 3);
+        if (n >= 4) a3 = al4(n - 4);
+    }
+    float4 x = ldg4(A.q + qrow * KDIM + lane * 4);
+    for (int i = n - 1; i >= 0; --i) {
+        const float4 kv = k0;
+        k0 = k1;
+        k1 = k2;
+        k2 = k3;
+        k3 = (i >= 4) ? kl(i - 4) : z;
+        float4 av = z;
+        if (KIND == SKETCHSSM_KDA) {
+            av = a0;
+            a0 = a1;
+            a1 = a2;
+            a2 = a3;
+            a3 = (i >= 4) ? al4(i - 4) : z;
+        }
+        const float bi = __shfl_sync(0xffffffffu, bl, i);
+        const float s1 = warp_sum(dot4(kv, x));
+        if (lane == 0) dst[rb + i] = bi * s1;
+        if (KIND == SKETCHSSM_GDN) {
+            const float ai = __shfl_sync(0xffffffffu, al, i);
+            const float t = bi * s1;
+            x.x = ai * fmaf(-t, kv.x, x.x);
+            x.y = ai * fmaf(-t, kv.y, x.y);
+            x.z = ai * fmaf(-t, kv.z, x.z);
+            x.w = ai * fmaf(-t, kv.w, x.w);
+        } else {
+            const float4 xa = make_float4(av.x * x.x, av.y * x.y, av.z * x.z, av.w * x.w);
+            const float t = bi * warp_sum(dot4(kv, xa));
+            x.x = fmaf(-t, kv.x, xa.x);
+            x.y = fmaf(-t, kv.y, xa.y);
+            x.z = fmaf(-t, kv.z, xa.z);
+            x.w = fmaf(-t, kv.w, xa.w);
+        }
+        if (i == pos) {
+            if (h == qk * hpq) st4(A.kbuf + (qrow * W + pos) * KDIM + lane * 4, kv);
+            if (KIND == SKETCHSSM_KDA) st4(A.abuf + (bh * W + pos) * KDIM + lane * 4, av);
+        }
+    }
+    // x = q0: base coefficients
+    if (dense) {
+        st4(dst + lane * 4, x);
+    } else {
+        const float *og = A.omega + (long long)g * A.Rb * KDIM + lane * 4;
+        for (int j0 = 0; j0 < rb; j0 += 8) {
+            float4 om[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) om[u] = (j0 + u < rb) ? ldg4(og + (long long)(j0 + u) * KDIM) : z;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (j0 + u >= rb) break;
+                const float d = warp_sum(dot4(om[u], x));
+                if (lane == 0) dst[j0 + u] = d;
+            }
+        }
+    }
+}
+
+// ============================================================================ combine
 
 struct Carve {
-    size_t hs, rstart, rbase, rneed, bptr, rinfo, coef, s, u, dp, q0, part, misc, total;
+    size_t bar, meta, coef, dots, qrow, as, stage, total;
 };
 
 __host__ __device__ inline size_t take(size_t &o, size_t bytes)
 {
-    size_t r = o;
-    o = (o + bytes + 15) & ~size_t(15);
+    const size_t r = o;
+    o = (o + bytes + 127) & ~size_t(127);
     return r;
 }
 
-__host__ __device__ inline Carve carve(int Hg, int W, int cap, int max_rows, int ns, int V)
+__host__ __device__ inline Carve carve(int kind, int stage_rows, int coef_cap, int V, int W, int maxnh,
+                                       int dots_row)
 {
+    const bool m2 = kind == SKETCHSSM_MAMBA2;
     Carve c;
     size_t o = 0;
-    c.hs = take(o, sizeof(int) * Hg);
-    c.rstart = take(o, sizeof(int) * (Hg + 1));
-    c.rbase = take(o, sizeof(int) * Hg);
-    c.rneed = take(o, sizeof(int) * Hg);
-    c.bptr = take(o, sizeof(long long) * Hg);
-    c.rinfo = take(o, sizeof(int) * max_rows);
-    c.coef = take(o, sizeof(float) * max_rows);
-    c.s = take(o, sizeof(float) * Hg * W);
-    c.u = take(o, sizeof(float) * Hg * cap);
-    c.dp = take(o, sizeof(float) * Hg);
-    c.q0 = take(o, sizeof(float) * Hg * KDIM);
-    c.part = take(o, sizeof(float) * (ns + Hg) * V);
-    c.misc = take(o, sizeof(int) * 4);
+    c.bar = take(o, 16);
+    c.meta = take(o, sizeof(int) * (6 * MAXC + 8));
+    c.coef = take(o, m2 ? 0 : sizeof(float) * (size_t)coef_cap);
+    c.dots = take(o, m2 ? sizeof(float) * (size_t)maxnh * dots_row : 0);
+    c.qrow = take(o, m2 ? sizeof(float) * KDIM : 0);
+    c.as = take(o, m2 ? sizeof(float) * (size_t)maxnh * W : 0);
+    c.stage = take(o, sizeof(float) * (size_t)stage_rows * V);
     c.total = o;
     return c;
 }
 
 template <int KIND>
-__global__ void __launch_bounds__(DECODE_MAX_THREADS)
-decode_kernel(const DecodeArgs A)
+__global__ void __launch_bounds__(256)
+combine_kernel(const DecodeArgs A)
 {
-    extern __shared__ __align__(16) unsigned char smem[];
-    const Carve cv = carve(A.Hg, A.W, A.cap, A.max_rows, A.ns, A.V);
-    int *hs = reinterpret_cast<int *>(smem + cv.hs);
-    int *rstart = reinterpret_cast<int *>(smem + cv.rstart);
-    int *rbase = reinterpret_cast<int *>(smem + cv.rbase);
-    int *rneed = reinterpret_cast<int *>(smem + cv.rneed);
-    long long *bptr = reinterpret_cast<long long *>(smem + cv.bptr);
-    int *rinfo = reinterpret_cast<int *>(smem + cv.rinfo);
+    constexpr bool M2 = KIND == SKETCHSSM_MAMBA2;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const Carve cv = carve(KIND, A.stage_rows, A.coef_cap, A.V, A.W, A.maxnh, A.dots_row);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + cv.bar);
+    int *meta = reinterpret_cast<int *>(smem + cv.meta);
+    int *hs = meta, *rb = meta + MAXC, *rbs = meta + 2 * MAXC, *cc = meta + 3 * MAXC, *ch = meta + 4 * MAXC;
     float *coef = reinterpret_cast<float *>(smem + cv.coef);
-    float *s_dot = reinterpret_cast<float *>(smem + cv.s);
-    float *u_dot = reinterpret_cast<float *>(smem + cv.u);
-    float *dpv = reinterpret_cast<float *>(smem + cv.dp);
-    float *q0s = reinterpret_cast<float *>(smem + cv.q0);
-    float *part = reinterpret_cast<float *>(smem + cv.part);
-    int *misc = reinterpret_cast<int *>(smem + cv.misc);
+    float *dots = reinterpret_cast<float *>(smem + cv.dots);
+    float *qrow_s = reinterpret_cast<float *>(smem + cv.qrow);
+    float *as_s = reinterpret_cast<float *>(smem + cv.as);
+    float *stage = reinterpret_cast<float *>(smem + cv.stage);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nwarps = blockDim.x >> 5;
     const int b = blockIdx.y;
-    const int item = A.dense_all ? -int(blockIdx.x) - 1 : A.work[blockIdx.x];
-    const bool dense = item < 0;
-    const int hd = -item - 1;                       // dense item: its head
-    const int g = dense ? hd / A.Hg : item;         // basis group
-    const int H = A.H, V = A.V, W = A.W, pos = A.pos, n = pos + 1;
-    const int Hg = A.Hg, hpq = A.hpq, Hqk = A.Hqk;
-    const int nch = dense ? 1 : Hg / hpq;          // q/k heads (chains) of a Mamba-2 item
-    const float *base = dense ? A.S : A.Y;
+    const int H = A.H, V = A.V, W = A.W, pos = A.pos, n = pos + 1, hpq = A.hpq, dr = A.dots_row;
+    // the item's record: {entry, span, member mask, rows R, off[h_first], coff[h_first], coef floats, h_first}
+    int R, yrow0, c0, cfl, h_first;
+    unsigned mask;
+    bool dense;
+    if (A.dense_all) {
+        dense = true;
+        h_first = blockIdx.x;
+        mask = 1u;
+        R = KDIM;
+        yrow0 = 0;
+        c0 = h_first * A.coef_dense_block;
+        cfl = A.coef_dense_block;
+    } else {
+        const int4 r0 = __ldg(reinterpret_cast<const int4 *>(A.rec) + 2 * blockIdx.x);
+        const int4 r1 = __ldg(reinterpret_cast<const int4 *>(A.rec) + 2 * blockIdx.x + 1);
+        dense = r0.x < 0;
+        mask = (unsigned)r0.z;
+        R = r0.w;
+        yrow0 = r1.x;
+        c0 = r1.y;
+        cfl = r1.z;
+        h_first = r1.w;
+    }
+    const int nh = __popc(mask);
 
-    // ------------------------------------------------------------ item set-up
     if (warp == 0) {
-        int h, rb;
-        bool member;
-        if (dense) {
-            h = hd;
-            member = lane == 0;
-            rb = KDIM;
-        } else {
-            h = g * Hg + lane;
-            const int r = (lane < Hg) ? __ldg(A.rank + h) : 0;
-            member = r > 0;
-            rb = r;
+        const int h = h_first + lane;
+        const bool member = (mask >> lane) & 1u;
+        const unsigned below = mask & ((1u << lane) - 1u);
+        const int slot = __popc(below);
+        // Mamba-2: the q/k heads (chains) of the members, in order
+        const int qk = h / hpq;
+        const int qk_prev = __shfl_sync(0xffffffffu, qk, below ? 31 - __clz(below) : lane);
+        const bool new_chain = M2 && member && (slot == 0 || qk != qk_prev);
+        const unsigned cmask = __ballot_sync(0xffffffffu, new_chain);
+        const int chain = __popc(cmask & ((2u << lane) - 1u)) - 1;
+        const int nch = __popc(cmask);
+        if (lane == 0) {
+            mbar_init(bar, 1);
+            mbar_fence_init();
+            uint32_t bytes = (uint32_t)((R + nh * n) * V * 4);
+            bytes += M2 ? (uint32_t)(nch * dr * 4 + (dense ? KDIM * 4 : 0)) : (uint32_t)(cfl * 4);
+            mbar_arrive_expect_tx(bar, bytes);
+            const float *src = dense ? A.S + ((long long)b * H + h_first) * KDIM * V
+                                     : A.Y + ((long long)b * A.rtot + yrow0) * V;
+            bulk_copy_g2s(stage, src, (uint32_t)(R * V * 4), bar);
+            if (M2 && dense) bulk_copy_g2s(qrow_s, A.q + ((long long)b * A.Hqk + qk) * KDIM, KDIM * 4, bar);
         }
-        const unsigned mask = __ballot_sync(0xffffffffu, member);
-        const int slot = __popc(mask & ((1u << lane) - 1u));
-        const int rows = member ? rb + n : 0;
-        int incl = rows;
+        __syncwarp();
+        const long long bh = (long long)b * H + h;
+        if (member) {
+            float *dst = stage + (size_t)(R + slot * n) * V;
+            if (pos > 0) bulk_copy_g2s(dst, A.vbuf + bh * W * V, (uint32_t)(pos * V * 4), bar);
+            bulk_copy_g2s(dst + (size_t)pos * V, A.v + bh * V, (uint32_t)(V * 4), bar);
+        }
+        // the products of the first launch of this step: wait until it has finished
+        pdl_wait_primary();
+        if (!M2 && lane == 0)
+            bulk_copy_g2s(coef, A.scratch + (long long)b * A.coef_row + c0, (uint32_t)(cfl * 4), bar);
+        if (new_chain)
+            bulk_copy_g2s(dots + (size_t)chain * dr, A.scratch + ((long long)b * A.Hqk + qk) * dr,
+                          (uint32_t)(dr * 4), bar);
+        // per-member layout (off the copies' path)
+        const int rbv = member ? (dense ? KDIM : __ldg(A.rank + h)) : 0;
+        int incl = rbv, cinc = member ? round4(rbv + W) : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
+            const int u = __shfl_up_sync(0xffffffffu, cinc, o);
+            if (lane >= o) {
+                incl += t;
+                cinc += u;
+            }
         }
-        if (lane < Hg) rneed[lane] = -1;
-        __syncwarp();
         if (member) {
             hs[slot] = h;
-            rbase[slot] = rb;
-            rstart[slot] = incl - rows;
-            bptr[slot] = dense ? ((long long)b * H + h) * KDIM * V
-                               : ((long long)b * A.rtot + __ldg(A.off + h)) * V;
-            if (KIND == SKETCHSSM_MAMBA2) atomicMax(&rneed[dense ? 0 : (h - g * Hg) / hpq], dense ? 0 : rb);
+            rb[slot] = rbv;
+            rbs[slot] = incl - rbv;
+            cc[slot] = cinc - round4(rbv + W);
+            ch[slot] = chain;
         }
-        if (lane == 31) {
-            const int nh = __popc(mask);
-            misc[0] = nh;
-            misc[1] = incl;
-            rstart[nh] = incl;
+    }
+    if (M2) {
+        // decays of the members' buffered tokens, spread over the CTA (one round of
+        // loads, in flight with the bulk copies); the step's decay goes to slot pos
+        for (int x = tid; x < nh * n; x += blockDim.x) {
+            const int slot = x / n, i = x - slot * n;
+            const long long bh = (long long)b * H + h_first + (int)__fns(mask, 0, slot + 1);
+            const float av = (i == pos) ? __ldg(A.a + bh) : __ldg(A.abuf + bh * W + i);
+            as_s[slot * W + i] = av;
+            if (i == pos) A.abuf[bh * W + pos] = av;
         }
     }
     __syncthreads();
-    const int nh = misc[0], total = misc[1];
-    for (int hl = warp; hl < nh; hl += nwarps) {
-        const int rows = rbase[hl] + n, r0 = rstart[hl];
-        for (int j = lane; j < rows; j += 32) rinfo[r0 + j] = (hl << 16) | j;
+    const bool ok = mbar_wait_bounded(bar, 0, A.wait_limit);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+            atomicOr(A.status, SK_STATUS_DECODE_TIMEOUT);
+            mbar_wait_bounded(bar, 0, A.wait_limit);  // a last chance for copies in flight
+        }
+        return;
     }
-
-    // ------------------------------------------------------------ phase A
-    if (KIND == SKETCHSSM_MAMBA2) {
-        // dot products of one warp each: chain c has n key dots and rneed[c] basis dots
-        const int cnt = (lane < nch && rneed[lane] >= 0) ? n + rneed[lane] : 0;
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const int start = incl - cnt;
-        const int ntask = __shfl_sync(0xffffffffu, incl, 31);
-        for (int t = warp; t < ntask; t += nwarps) {
-            const unsigned hit = __ballot_sync(0xffffffffu, cnt > 0 && start <= t && t < start + cnt);
-            const int c = __ffs(hit) - 1;
-            const int idx = t - __shfl_sync(0xffffffffu, start, c);
-            const int qk = dense ? hd / hpq : (g * Hg) / hpq + c;
-            const long long qrow = (long long)b * Hqk + qk;
-            const float4 qv = ldg4(A.q + qrow * KDIM + lane * 4);
-            float4 vec;
-            if (idx < n) {
-                vec = (idx == pos) ? ldg4(A.k + qrow * KDIM + lane * 4)
-                                   : ldg4(A.kbuf + (qrow * W + idx) * KDIM + lane * 4);
-            } else {
-                vec = ldg4(A.omega + ((long long)g * A.Rb + (idx - n)) * KDIM + lane * 4);
-            }
-            const float d = warp_sum(dot4(qv, vec));
-            if (lane == 0) {
-                if (idx < n) s_dot[c * W + idx] = d;
-                else u_dot[c * A.cap + (idx - n)] = d;
-            }
-            if (idx == pos) {
-                // this item writes the key if it handles the first head of the q/k head
-                const int h0 = qk * hpq;
-                const bool owner = dense ? (hd == h0) : (__ldg(A.rank + h0) > 0);
-                if (owner) st4(A.kbuf + (qrow * W + pos) * KDIM + lane * 4, vec);
-            }
-        }
-        __syncthreads();
-        if (tid < nh) {
-            const int h = hs[tid];
-            const int c = dense ? 0 : (h - g * Hg) / hpq;
-            const long long bh = (long long)b * H + h;
-            const int r0 = rstart[tid] + rbase[tid];
-            float dp = 1.f;
-            for (int i = n - 1; i >= 0; --i) {
-                const float ai = (i == pos) ? __ldg(A.a + bh) : __ldg(A.abuf + bh * W + i);
-                coef[r0 + i] = dp * s_dot[c * W + i];
-                dp *= ai;
-            }
-            dpv[tid] = dp;
-            A.abuf[bh * W + pos] = __ldg(A.a + bh);
-        }
-        __syncthreads();
-        for (int e = tid; e < total; e += blockDim.x) {
-            const int info = rinfo[e], hl = info >> 16, j = info & 0xffff;
-            if (j >= rbase[hl]) continue;
-            if (dense) {
-                coef[e] = dpv[0] * __ldg(A.q + ((long long)b * Hqk + hd / hpq) * KDIM + j);
-            } else {
-                const int c = (hs[hl] - g * Hg) / hpq;
-                coef[e] = dpv[hl] * u_dot[c * A.cap + j];
-            }
-        }
-    } else {
-        // GDN / KDA: one warp per head walks the buffer newest first
-        for (int hl = warp; hl < nh; hl += nwarps) {
-            const int h = hs[hl], qk = h / hpq;
-            const long long bh = (long long)b * H + h;
-            const long long qrow = (long long)b * Hqk + qk;
-            float4 x = ldg4(A.q + qrow * KDIM + lane * 4);
-            const int r0 = rstart[hl] + rbase[hl];
-            for (int i = n - 1; i >= 0; --i) {
-                const bool cur = (i == pos);
-                const float4 kv = cur ? ldg4(A.k + qrow * KDIM + lane * 4)
-                                      : ldg4(A.kbuf + (qrow * W + i) * KDIM + lane * 4);
-                const float bi = cur ? __ldg(A.beta + bh) : __ldg(A.bbuf + bh * W + i);
-                const float s1 = warp_sum(dot4(kv, x));
-                if (lane == 0) coef[r0 + i] = bi * s1;
-                if (KIND == SKETCHSSM_GDN) {
-                    const float ai = cur ? __ldg(A.a + bh) : __ldg(A.abuf + bh * W + i);
-                    const float t = bi * s1;
-                    x.x = ai * fmaf(-t, kv.x, x.x);
-                    x.y = ai * fmaf(-t, kv.y, x.y);
-                    x.z = ai * fmaf(-t, kv.z, x.z);
-                    x.w = ai * fmaf(-t, kv.w, x.w);
-                    if (cur && lane == 0) A.abuf[bh * W + pos] = ai;
-                } else {
-                    const float4 av = cur ? ldg4(A.a + bh * KDIM + lane * 4)
-                                          : ldg4(A.abuf + (bh * W + i) * KDIM + lane * 4);
-                    const float4 xa = make_float4(av.x * x.x, av.y * x.y, av.z * x.z, av.w * x.w);
-                    const float t = bi * warp_sum(dot4(kv, xa));
-                    x.x = fmaf(-t, kv.x, xa.x);
-                    x.y = fmaf(-t, kv.y, xa.y);
-                    x.z = fmaf(-t, kv.z, xa.z);
-                    x.w = fmaf(-t, kv.w, xa.w);
-                    if (cur) st4(A.abuf + (bh * W + pos) * KDIM + lane * 4, av);
-                }
-                if (cur) {
-                    if (h == qk * hpq) st4(A.kbuf + (qrow * W + pos) * KDIM + lane * 4, kv);
-                    if (lane == 0) A.bbuf[bh * W + pos] = bi;
-                }
-            }
-            st4(q0s + hl * KDIM + lane * 4, x);
-        }
-        __syncthreads();
-        if (dense) {
-            for (int j = tid; j < KDIM; j += blockDim.x) coef[j] = q0s[j];
-        } else {
-            for (int e = warp; e < total; e += nwarps) {
-                const int info = rinfo[e], hl = info >> 16, j = info & 0xffff;
-                if (j >= rbase[hl]) continue;  // warp-uniform
-                const float4 om = ldg4(A.omega + ((long long)g * A.Rb + j) * KDIM + lane * 4);
-                const float d = warp_sum(dot4(om, lds4(q0s + hl * KDIM + lane * 4)));
-                if (lane == 0) coef[e] = d;
-            }
-        }
-    }
-    __syncthreads();
-
-    // ------------------------------------------------------------ phase B
     const int V4 = V >> 2;
-    const int ns = A.ns;
-    const int chunk = (total + ns - 1) / ns;
-    const int sl = tid / V4, c4 = tid - sl * V4;
-    if (sl < ns) {
-        const int e0 = sl * chunk;
-        const int e1 = min(e0 + chunk, total);
-        float4 acc = zero4();
-        int curh = -1;
-        for (int e = e0; e < e1; e += UNROLL) {
-            float4 xv[UNROLL];
-            float cf[UNROLL];
-            int hv[UNROLL];
-            float *app[UNROLL];
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                hv[u] = -1;
-                app[u] = nullptr;
-                const int ee = e + u;
-                if (ee < e1) {
-                    const int info = rinfo[ee], hl = info >> 16, j = info & 0xffff;
-                    const int rb = rbase[hl];
-                    const float *src;
-                    if (j < rb) {
-                        src = base + bptr[hl] + (long long)j * V;
-                    } else {
-                        const int i = j - rb;
-                        const long long bh = (long long)b * H + hs[hl];
-                        if (i == pos) {
-                            src = A.v + bh * V;
-                            app[u] = A.vbuf + (bh * W + pos) * V + c4 * 4;
-                        } else {
-                            src = A.vbuf + (bh * W + i) * V;
-                        }
-                    }
-                    xv[u] = ldg4(src + c4 * 4);
-                    cf[u] = coef[ee];
-                    hv[u] = hl;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u)
-                if (app[u]) st4(app[u], xv[u]);
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                if (hv[u] < 0) continue;
-                if (hv[u] != curh) {
-                    if (curh >= 0) st4(part + (sl + curh) * V + c4 * 4, acc);
-                    acc = zero4();
-                    curh = hv[u];
-                }
-                fma4(acc, cf[u], xv[u]);
-            }
-        }
-        if (curh >= 0) st4(part + (sl + curh) * V + c4 * 4, acc);
-    }
-    __syncthreads();
     for (int o = tid; o < nh * V4; o += blockDim.x) {
-        const int hl = o / V4, cc = o - hl * V4;
-        const int s0 = rstart[hl] / chunk, s1 = (rstart[hl + 1] - 1) / chunk;
-        float4 sum = zero4();
-        for (int s = s0; s <= s1; ++s) {
-            const float4 p = lds4(part + (s + hl) * V + cc * 4);
-            sum.x += p.x;
-            sum.y += p.y;
-            sum.z += p.z;
-            sum.w += p.w;
+        const int hl = o / V4, c4 = o - hl * V4;
+        const int r0 = rbs[hl], rbh = rb[hl], rr = R + hl * n;
+        const float *sp = stage + c4 * 4;
+        float4 acc0 = zero4(), acc1 = zero4();
+        if (M2) {
+            const float *sv = dots + (size_t)ch[hl] * dr;
+            const float *uv = dense ? qrow_s : sv + W;
+            const float *av = as_s + hl * W;
+            float w = 1.f;  // prod_{j>i} a_j, newest token first; ends as decay_prod
+            for (int i = n - 1; i >= 0; --i) {
+                fma4(acc1, w * sv[i], lds4(sp + (size_t)(rr + i) * V));
+                w *= av[i];
+            }
+            int j = 0;
+            for (; j + 1 < rbh; j += 2) {
+                fma4(acc0, w * uv[j], lds4(sp + (size_t)(r0 + j) * V));
+                fma4(acc1, w * uv[j + 1], lds4(sp + (size_t)(r0 + j + 1) * V));
+            }
+            if (j < rbh) fma4(acc0, w * uv[j], lds4(sp + (size_t)(r0 + j) * V));
+        } else {
+            const float *cf = coef + cc[hl];
+            int j = 0;
+            for (; j + 1 < rbh; j += 2) {
+                fma4(acc0, cf[j], lds4(sp + (size_t)(r0 + j) * V));
+                fma4(acc1, cf[j + 1], lds4(sp + (size_t)(r0 + j + 1) * V));
+            }
+            if (j < rbh) fma4(acc0, cf[j], lds4(sp + (size_t)(r0 + j) * V));
+            for (int i = 0; i < n; ++i) fma4(acc1, cf[rbh + i], lds4(sp + (size_t)(rr + i) * V));
         }
-        st4(A.y + ((long long)b * H + hs[hl]) * V + cc * 4, sum);
+        const float4 acc = make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
+        const long long bh = (long long)b * H + hs[hl];
+        st4(A.y + bh * V + c4 * 4, acc);
+        st4(A.vbuf + (bh * W + pos) * V + c4 * 4, lds4(sp + (size_t)(rr + pos) * V));
     }
 }
 
 template <int KIND>
-cudaError_t launch_kind(const DecodeArgs &a, cudaStream_t stream)
+cudaError_t launch_combine(const DecodeArgs &a, cudaStream_t stream)
 {
-    int ns = 0;
-    const int threads = decode_threads(a.V, &ns);
     const size_t smem = decode_smem_bytes(a);
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<KIND>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(combine_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(a.dense_all ? a.H : a.n_work, a.B);
-    decode_kernel<KIND><<<grid, threads, smem, stream>>>(a);
+    // programmatic dependent launch: CTAs may start while the products kernel runs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.n_items, a.B);
+    cfg.blockDim = dim3(a.threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, combine_kernel<KIND>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int decode_threads(int V, int *ns_out)
+int dots_row(int W, int cap) { return round4(W + cap); }
+
+bool decode_geometry(int kind, int V, int W, int cap, int Hg, DecodeGeometry *gm)
 {
     const int V4 = V / 4;
-    int ns = DECODE_THREADS_TARGET / V4;
-    if (ns < 1) ns = 1;
-    if (ns_out) *ns_out = ns;
-    return ((ns * V4 + 31) / 32) * 32;
+    // items may hold a whole group: the row budget bounds their bytes, and the row sums
+    // loop over (head, column chunk) outputs when they outnumber the threads
+    const int m = Hg < MAXC ? Hg : MAXC;
+    gm->maxnh = m;
+    int per = COMBINE_TARGET_THREADS / V4;
+    if (per < 1) per = 1;
+    if (per > m) per = m;
+    int t = ((per * V4 + 31) / 32) * 32;
+    if (t < 64) t = 64;
+    if (t > 256) t = 256;
+    gm->threads = t;
+    int rows = STAGE_TARGET / (4 * V);
+    if (rows < KDIM + W) rows = KDIM + W;
+    if (rows < cap + W) rows = cap + W;
+    gm->stage_rows = rows;
+    gm->coef_cap = rows + m * (W + 3) + 4;
+    return carve(kind, rows, gm->coef_cap, V, W, m, dots_row(W, cap)).total <= 227 * 1024 &&
+           cm_carve(cap, W, 1).total <= 227 * 1024;
+}
+
+int coef_block(int rows, int W) { return round4(rows + W); }
+
+int coef_rows(int cap, int W)
+{
+    // batch rows per Mamba-2 product CTA: as many as keep two CTAs on an SM
+    for (int rows = CM_MAXROWS; rows > 1; rows >>= 1)
+        if (cm_carve(cap, W, rows).total <= 110 * 1024) return rows;
+    return 1;
 }
 
 size_t decode_smem_bytes(const DecodeArgs &a)
 {
-    return carve(a.Hg, a.W, a.cap, a.max_rows, a.ns, a.V).total;
+    return carve(a.kind, a.stage_rows, a.coef_cap, a.V, a.W, a.maxnh, a.dots_row).total;
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream)
 {
-    if (a.B == 0 || (a.dense_all ? a.H : a.n_work) == 0) return cudaSuccess;
+    if (a.B == 0) return cudaSuccess;
+    cudaError_t e;
+    if (a.kind == SKETCHSSM_MAMBA2) {
+        const size_t cm = cm_carve(a.cap, a.W, a.cm_rows).total;
+        if ((e = cudaFuncSetAttribute(dots_kernel_mamba2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cm)) !=
+            cudaSuccess)
+            return e;
+        dots_kernel_mamba2<<<dim3(a.Hqk, (a.B + a.cm_rows - 1) / a.cm_rows), CM_THREADS, cm, stream>>>(a);
+    } else {
+        const dim3 grid((a.H + COEF_THREADS / 32 - 1) / (COEF_THREADS / 32), a.B);
+        if (a.kind == SKETCHSSM_GDN) coef_kernel_delta<SKETCHSSM_GDN><<<grid, COEF_THREADS, 0, stream>>>(a);
+        else coef_kernel_delta<SKETCHSSM_KDA><<<grid, COEF_THREADS, 0, stream>>>(a);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.n_items == 0) return cudaSuccess;
     switch (a.kind) {
-    case SKETCHSSM_MAMBA2: return launch_kind<SKETCHSSM_MAMBA2>(a, stream);
-    case SKETCHSSM_GDN: return launch_kind<SKETCHSSM_GDN>(a, stream);
-    default: return launch_kind<SKETCHSSM_KDA>(a, stream);
+    case SKETCHSSM_MAMBA2: return launch_combine<SKETCHSSM_MAMBA2>(a, stream);
+    case SKETCHSSM_GDN: return launch_combine<SKETCHSSM_GDN>(a, stream);
+    default: return launch_combine<SKETCHSSM_KDA>(a, stream);
     }
 }
 

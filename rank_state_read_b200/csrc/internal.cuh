@@ -11,22 +11,40 @@
 namespace sk {
 
 constexpr int KDIM = 128;        // key dim the kernels are built for (Nemotron Nano card)
-constexpr int KDIM4 = KDIM / 4;  // float4 lanes of a key vector: one per warp lane
 constexpr int MAX_HG = 32;       // heads per basis group
 constexpr int MAX_W = 32;        // buffer window
 constexpr int MAX_V = 256;       // value dim
 
-// Arguments of one decode launch (sketch or dense-read).
+// bits of the plan's device status word
+constexpr int SK_STATUS_DECODE_TIMEOUT = 1;
+
+// default bound of a kernel's wait on its own bulk copies (clock cycles, ~1 s)
+constexpr long long DEFAULT_WAIT_CYCLES = 2000000000LL;
+
+// Arguments of one decode step (sketch or dense-read): coefficient + combine launches.
 struct DecodeArgs {
     int kind, B, H, Hqk, V, W, G, Rb, cap, pos;
-    int Hg;        // heads per group
-    int hpq;       // heads per q/k head
-    int64_t rtot;  // sketch rows per batch row
-    const int *rank, *off, *work;
-    int n_work;    // items per batch row
-    int dense_all; // 1: every head is a dense item (dense-read baseline)
-    int ns;        // row slices of the weighted row sum
-    int max_rows;  // capacity of the per-item row tables
+    int Hg;              // heads per group
+    int hpq;             // heads per q/k head
+    int64_t rtot;        // sketch rows per batch row
+    const int *rank, *off;
+    const int *coff;     // coefficient block of each head within a batch row (sketch layout)
+    int coef_row;        // coefficient floats per batch row (of the layout in use)
+    int coef_dense_block;// per-head block of the dense-read layout (head h at h * block)
+    float *scratch;      // Mamba-2: products, B x Hqk x dots_row; GDN/KDA: coefficients, B x coef_row
+    const int *work;     // combine items of this step (already offset to its n)
+    const int *rec;      // their records, 8 ints each (layout kernel)
+    const int *qk_rneed; // largest sketch rank per q/k head
+    int n_items;         // combine items per batch row
+    int dense_all;       // 1: every head reads its state (dense-read baseline)
+    int threads;         // combine CTA size
+    int stage_rows;      // rows of the combine stage
+    int cm_rows;         // batch rows per Mamba-2 product CTA
+    int dots_row;        // Mamba-2 products per (batch row, q/k head): W keys, then cap basis rows
+    int maxnh;           // heads per combine item at most
+    int coef_cap;        // floats of the combine coefficient stage
+    long long wait_limit;
+    int *status;
     const float *q, *k, *v, *a, *beta;
     float *kbuf, *vbuf, *abuf, *bbuf;
     const float *Y, *omega, *S;
@@ -37,6 +55,7 @@ struct DecodeArgs {
 struct FlushArgs {
     int kind, B, H, Hqk, V, W, G, Rb, cap, n;
     int Hg, hpq;
+    int VS;  // column slab of one work item
     int64_t rtot;
     const int *rank, *off;
     float *S;
@@ -44,18 +63,28 @@ struct FlushArgs {
     float *Y;
 };
 
-// Dynamic shared memory of a decode CTA (bytes) and its thread count.
+// Geometry of the combine launch for a layer shape: heads per item, CTA size, rows of
+// one shared-memory stage (the packing budget of a sketch item), coefficient stage.
+struct DecodeGeometry {
+    int maxnh, threads, stage_rows, coef_cap;
+};
+bool decode_geometry(int kind, int V, int W, int cap, int Hg, DecodeGeometry *gm);
+int coef_block(int rows, int W);  // floats of one head's coefficient block
+int coef_rows(int cap, int W);
+int dots_row(int W, int cap);
 size_t decode_smem_bytes(const DecodeArgs &a);
-int decode_threads(int V, int *ns_out);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
-size_t flush_smem_bytes(int kind, int V, int W, int cap);
-int flush_threads(int V);
+int flush_slab(int V);
+size_t flush_smem_bytes(int kind, int V, int W);
 cudaError_t launch_flush(const FlushArgs &a, cudaStream_t stream);
 
-// Layout kernel: off[H+1], rmax[G], work[G+H]; counts = {n_work, n_dense, err, max_group_rows}.
-cudaError_t launch_layout(const int *rank, int H, int G, int cap, int *off, int *rmax, int *work,
-                          int *counts, cudaStream_t stream);
+// Layout kernel: off[H+1], rmax[G], coff[H], per-n work lists work[(n-1)(H+G) ...];
+// counts = {dense heads, invalid-rank flag, coefficient floats per row, items for
+// n = 1 .. W}.
+cudaError_t launch_layout(const int *rank, int H, int G, int Hqk, int W, int cap, int row_budget, int max_heads,
+                          int *off, int *rmax, int *coff, int *work, int *rec, int *qk_rneed, int *counts,
+                          cudaStream_t stream);
 
 }  // namespace sk
 
@@ -63,8 +92,13 @@ struct sketchssm_plan {
     sketchssm_desc d;
     int Hg, hpq;
     int64_t rtot;
-    int n_work, n_dense, max_group_rows;
+    int n_dense;
+    sk::DecodeGeometry geo;
     int device;
-    int *d_rank, *d_off, *d_rmax, *d_work, *d_counts;
-    std::vector<int32_t> h_rank, h_off, h_rmax, h_work;
+    long long wait_limit;
+    int coef_row;
+    int *d_rank, *d_off, *d_rmax, *d_coff, *d_work, *d_rec, *d_qk_rneed, *d_counts, *d_status;
+    float *d_scratch;
+    size_t scratch_floats;
+    std::vector<int32_t> h_rank, h_off, h_rmax, h_work, h_items;
 };

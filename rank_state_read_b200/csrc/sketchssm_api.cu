@@ -149,13 +149,23 @@ sk::DecodeArgs decode_args(const sketchssm_plan *p, int pos, const float *q, con
     A.rtot = p->rtot;
     A.rank = p->d_rank;
     A.off = p->d_off;
-    A.work = p->d_work;
-    A.n_work = p->n_work;
+    A.coff = p->d_coff;
+    A.coef_dense_block = sk::coef_block(sk::KDIM, d.window);
+    A.coef_row = dense_all ? d.heads * A.coef_dense_block : p->coef_row;
+    A.scratch = p->d_scratch;
+    A.work = p->d_work + (size_t)pos * (d.heads + d.groups);
+    A.rec = p->d_rec + (size_t)pos * (d.heads + d.groups) * 8;
+    A.qk_rneed = p->d_qk_rneed;
+    A.n_items = dense_all ? d.heads : p->h_items[pos];
     A.dense_all = dense_all;
-    sk::decode_threads(d.value_dim, &A.ns);
-    const int grp = p->max_group_rows + p->Hg * d.window;
-    const int den = sk::KDIM + d.window;
-    A.max_rows = grp > den ? grp : den;
+    A.threads = p->geo.threads;
+    A.stage_rows = p->geo.stage_rows;
+    A.cm_rows = sk::coef_rows(d.rank_cap, d.window);
+    A.dots_row = sk::dots_row(d.window, d.rank_cap);
+    A.maxnh = p->geo.maxnh;
+    A.coef_cap = p->geo.coef_cap;
+    A.wait_limit = p->wait_limit;
+    A.status = p->d_status;
     A.q = q;
     A.k = k;
     A.v = v;
@@ -241,47 +251,72 @@ sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t
     p->d = d;
     p->Hg = H / G;
     p->hpq = H / d.qk_heads;
+    p->wait_limit = sk::DEFAULT_WAIT_CYCLES;
+    if (!sk::decode_geometry(d.kind, d.value_dim, d.window, d.rank_cap, p->Hg, &p->geo)) {
+        delete p;
+        return fail(SKETCHSSM_ERR_UNSUPPORTED, "a decode work item of this shape does not fit in shared memory");
+    }
     cudaGetDevice(&p->device);
-    p->d_rank = p->d_off = p->d_rmax = p->d_work = p->d_counts = nullptr;
+    p->d_rank = p->d_off = p->d_rmax = p->d_coff = p->d_work = p->d_rec = p->d_qk_rneed = nullptr;
+    p->d_counts = p->d_status = nullptr;
+    p->d_scratch = nullptr;
     cudaStream_t st = (cudaStream_t)stream;
     auto bail = [&](cudaError_t e, const char *what) {
         sketchssm_plan_destroy(p);
         return cuda_fail(e, what);
     };
+    const int W = d.window;
+    const size_t stride = (size_t)H + G;
     cudaError_t e;
     if ((e = cudaMalloc(&p->d_rank, sizeof(int) * H)) != cudaSuccess) return bail(e, "cudaMalloc");
     if ((e = cudaMalloc(&p->d_off, sizeof(int) * (H + 1))) != cudaSuccess) return bail(e, "cudaMalloc");
     if ((e = cudaMalloc(&p->d_rmax, sizeof(int) * G)) != cudaSuccess) return bail(e, "cudaMalloc");
-    if ((e = cudaMalloc(&p->d_work, sizeof(int) * (G + H))) != cudaSuccess) return bail(e, "cudaMalloc");
-    if ((e = cudaMalloc(&p->d_counts, sizeof(int) * 4)) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_coff, sizeof(int) * H)) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_work, sizeof(int) * stride * W)) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_rec, sizeof(int) * 8 * stride * W)) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_qk_rneed, sizeof(int) * d.qk_heads)) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_counts, sizeof(int) * (3 + W))) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMalloc(&p->d_status, sizeof(int))) != cudaSuccess) return bail(e, "cudaMalloc");
+    if ((e = cudaMemsetAsync(p->d_status, 0, sizeof(int), st)) != cudaSuccess) return bail(e, "cudaMemsetAsync");
     if ((e = cudaMemcpyAsync(p->d_rank, rank_host, sizeof(int) * H, cudaMemcpyHostToDevice, st)) !=
         cudaSuccess)
         return bail(e, "cudaMemcpyAsync(rank)");
-    if ((e = sk::launch_layout(p->d_rank, H, G, d.rank_cap, p->d_off, p->d_rmax, p->d_work,
-                               p->d_counts, st)) != cudaSuccess)
+    if ((e = sk::launch_layout(p->d_rank, H, G, d.qk_heads, W, d.rank_cap, p->geo.stage_rows, p->geo.maxnh,
+                               p->d_off, p->d_rmax, p->d_coff, p->d_work, p->d_rec, p->d_qk_rneed, p->d_counts,
+                               st)) != cudaSuccess)
         return bail(e, "layout kernel launch");
-    int counts[4];
+    std::vector<int> counts(3 + W);
     p->h_off.resize(H + 1);
     p->h_rmax.resize(G);
-    p->h_work.resize(G + H);
-    if ((e = cudaMemcpyAsync(counts, p->d_counts, sizeof(counts), cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+    p->h_work.resize(stride * W);
+    if ((e = cudaMemcpyAsync(counts.data(), p->d_counts, sizeof(int) * (3 + W), cudaMemcpyDeviceToHost, st)) !=
+            cudaSuccess ||
         (e = cudaMemcpyAsync(p->h_off.data(), p->d_off, sizeof(int) * (H + 1), cudaMemcpyDeviceToHost, st)) !=
             cudaSuccess ||
         (e = cudaMemcpyAsync(p->h_rmax.data(), p->d_rmax, sizeof(int) * G, cudaMemcpyDeviceToHost, st)) !=
             cudaSuccess ||
-        (e = cudaMemcpyAsync(p->h_work.data(), p->d_work, sizeof(int) * (G + H), cudaMemcpyDeviceToHost,
+        (e = cudaMemcpyAsync(p->h_work.data(), p->d_work, sizeof(int) * stride * W, cudaMemcpyDeviceToHost,
                              st)) != cudaSuccess)
         return bail(e, "cudaMemcpyAsync(layout)");
     if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return bail(e, "layout kernel");
-    if (counts[2] != 0) {
+    if (counts[1] != 0) {
         sketchssm_plan_destroy(p);
         return fail(SKETCHSSM_ERR_INVALID_ARG, "layout kernel found an invalid rank");
     }
-    p->n_work = counts[0];
-    p->n_dense = counts[1];
-    p->max_group_rows = counts[3];
+    p->n_dense = counts[0];
+    p->coef_row = counts[2];
+    p->h_items.assign(counts.begin() + 3, counts.end());
+    {
+        // coefficient scratch: the sketch layout, or the dense-read layout, per batch row
+        const size_t dense_row = (size_t)H * sk::coef_block(sk::KDIM, W);
+        size_t row = (size_t)p->coef_row > dense_row ? (size_t)p->coef_row : dense_row;
+        const size_t dots = (size_t)d.qk_heads * sk::dots_row(W, d.rank_cap);
+        if (dots > row) row = dots;
+        p->scratch_floats = row * (size_t)d.batch;
+        if ((e = cudaMalloc(&p->d_scratch, sizeof(float) * p->scratch_floats)) != cudaSuccess)
+            return bail(e, "cudaMalloc(coefficient scratch)");
+    }
     p->rtot = p->h_off[H];
-    p->h_work.resize(p->n_work);
     p->h_rank.assign(rank_host, rank_host + H);
     if (p->rtot != rtot) {
         sketchssm_plan_destroy(p);
@@ -292,15 +327,40 @@ sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t
 }
 
 sketchssm_status sketchssm_plan_query(const sketchssm_plan *p, int64_t *r_total, int32_t *offsets_host,
-                                      int32_t *rmax_host, int32_t *work_host, int32_t *n_work)
+                                      int32_t *rmax_host, int32_t n_tokens, int32_t *work_host,
+                                      int32_t *n_work)
 {
     g_last_error.clear();
     if (!p) return fail(SKETCHSSM_ERR_INVALID_ARG, "plan is NULL");
     if (r_total) *r_total = p->rtot;
     if (offsets_host) std::memcpy(offsets_host, p->h_off.data(), sizeof(int32_t) * p->h_off.size());
     if (rmax_host) std::memcpy(rmax_host, p->h_rmax.data(), sizeof(int32_t) * p->h_rmax.size());
-    if (work_host) std::memcpy(work_host, p->h_work.data(), sizeof(int32_t) * p->h_work.size());
-    if (n_work) *n_work = p->n_work;
+    if (!work_host && !n_work) return SKETCHSSM_OK;
+    const size_t stride = (size_t)p->d.heads + p->d.groups;
+    if (n_tokens < 1 || n_tokens > p->d.window)
+        return fail(SKETCHSSM_ERR_INVALID_ARG, "n_tokens outside [1, window]");
+    const int items = p->h_items[n_tokens - 1];
+    if (work_host)
+        std::memcpy(work_host, p->h_work.data() + (size_t)(n_tokens - 1) * stride, sizeof(int32_t) * items);
+    if (n_work) *n_work = items;
+    return SKETCHSSM_OK;
+}
+
+sketchssm_status sketchssm_plan_check(const sketchssm_plan *p, sketchssm_stream stream)
+{
+    g_last_error.clear();
+    sketchssm_status s = check_plan(p);
+    if (s != SKETCHSSM_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    int flags = 0;
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(&flags, p->d_status, sizeof(int), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpyAsync(status)");
+    if ((e = cudaMemsetAsync(p->d_status, 0, sizeof(int), st)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemsetAsync(status)");
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream");
+    if (flags & sk::SK_STATUS_DECODE_TIMEOUT)
+        return fail(SKETCHSSM_ERR_TIMEOUT, "a decode CTA gave up waiting for its bulk copies; its outputs are incomplete");
     return SKETCHSSM_OK;
 }
 
@@ -310,8 +370,13 @@ sketchssm_status sketchssm_plan_destroy(sketchssm_plan *p)
     cudaFree(p->d_rank);
     cudaFree(p->d_off);
     cudaFree(p->d_rmax);
+    cudaFree(p->d_coff);
     cudaFree(p->d_work);
+    cudaFree(p->d_rec);
+    cudaFree(p->d_qk_rneed);
+    cudaFree(p->d_scratch);
     cudaFree(p->d_counts);
+    cudaFree(p->d_status);
     delete p;
     return SKETCHSSM_OK;
 }
@@ -350,6 +415,7 @@ sketchssm_status sketchssm_flush(const sketchssm_plan *p, float *S, const float 
     A.n = n_tokens;
     A.Hg = p->Hg;
     A.hpq = p->hpq;
+    A.VS = sk::flush_slab(d.value_dim);
     A.rtot = p->rtot;
     A.rank = p->d_rank;
     A.off = p->d_off;
@@ -381,8 +447,6 @@ sketchssm_status sketchssm_decode(const sketchssm_plan *p, int32_t pos, const fl
     CHECK_T(omega, any_sketch ? fbytes(d.groups, d.basis_rows, d.key_dim) : 0, "omega", !any_sketch);
     CHECK_T(S, any_dense ? fbytes(d.batch, d.heads, d.key_dim, d.value_dim) : 0, "S", !any_dense);
     const sk::DecodeArgs A = decode_args(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, Y, omega, S, y, 0);
-    if (sk::decode_smem_bytes(A) > 200 * 1024)
-        return fail(SKETCHSSM_ERR_UNSUPPORTED, "decode item needs more than 200 KB of shared memory");
     cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     return SKETCHSSM_OK;
@@ -401,8 +465,6 @@ sketchssm_status sketchssm_dense_decode(const sketchssm_plan *p, int32_t pos, co
     const sketchssm_desc &d = p->d;
     CHECK_T(S, fbytes(d.batch, d.heads, d.key_dim, d.value_dim), "S", false);
     const sk::DecodeArgs A = decode_args(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, nullptr, nullptr, S, y, 1);
-    if (sk::decode_smem_bytes(A) > 200 * 1024)
-        return fail(SKETCHSSM_ERR_UNSUPPORTED, "decode item needs more than 200 KB of shared memory");
     cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "dense decode kernel launch");
     return SKETCHSSM_OK;

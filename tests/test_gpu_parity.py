@@ -47,8 +47,44 @@ def layout_tables():
         r = rng.integers(1, cfg.cap + 1, cfg.H).astype(np.int32)
         r[rng.random(cfg.H) < 0.3] = DENSE
         out.append((f"random{i}", cfg, r))
+    out.append(("mamba2-per-head-qk", cfg.replace(Hqk=cfg.H), synth.layer_rank_table(cfg)))
     out.append(("all-dense", cfg, np.full(cfg.H, DENSE, np.int32)))
     out.append(("all-cap", cfg, np.full(cfg.H, cfg.cap, np.int32)))
+    return out
+
+
+def decode_geometry(cfg):
+    """Item limits of the combine launch: heads per item and rows of one stage."""
+    maxnh = min(32, cfg.H // cfg.G)
+    rows = max(40 * 1024 // (4 * cfg.V), cfg.K + cfg.W, cfg.cap + cfg.W)
+    return maxnh, rows
+
+
+def item_cost(cfg, rank, heads, n):
+    return sum(int(rank[h]) + n for h in heads)
+
+
+def expected_work(rank, cfg):
+    """Definition of the per-n work lists: dense heads first (head order), then per group
+    the sketch heads packed greedily in head order while their rows (r + n) fit."""
+    maxnh, budget = decode_geometry(cfg)
+    H, G, Hg = cfg.H, cfg.G, cfg.H // cfg.G
+    dense = [-h - 1 for h in range(H) if rank[h] == DENSE]
+    out = {}
+    for n in range(1, cfg.W + 1):
+        items = list(dense)
+        for g in range(G):
+            cur = []
+            for h in range(g * Hg, (g + 1) * Hg):
+                if rank[h] <= 0:
+                    continue
+                if cur and (item_cost(cfg, rank, cur + [h], n) > budget or len(cur) == maxnh):
+                    items.append(cur[0] * 64 + cur[-1] - cur[0] + 1)
+                    cur = []
+                cur.append(h)
+            if cur:
+                items.append(cur[0] * 64 + cur[-1] - cur[0] + 1)
+        out[n] = items
     return out
 
 
@@ -61,10 +97,18 @@ def test_layout_bit_exact(name, cfg, rank):
     assert plan.offsets == off.tolist()
     assert plan.rmax == rmax.tolist()
     assert plan.r_total == rtot
-    Hg = cfg.H // cfg.G
-    expect = [-h - 1 for h in range(cfg.H) if rank[h] == DENSE]
-    expect += [g for g in range(cfg.G) if (rank[g * Hg:(g + 1) * Hg] > 0).any()]
-    assert plan.work == expect
+    assert plan.work == expected_work(rank, cfg)
+    # every sketch head lands in exactly one item of each list, within the stage budget
+    _, budget = decode_geometry(cfg)
+    for n, items in plan.work.items():
+        seen = []
+        for e in items:
+            if e < 0:
+                continue
+            hs = [h for h in range(e // 64, e // 64 + e % 64) if rank[h] > 0]
+            assert item_cost(cfg, rank, hs, n) <= budget
+            seen += hs
+        assert sorted(seen) == [h for h in range(cfg.H) if rank[h] > 0]
     plan.close()
 
 
@@ -127,11 +171,19 @@ def test_shared_qk_gdn():
     parity_run(small(3, B=2, Hqk=4), 18)
 
 
-@pytest.mark.parametrize("V,W,H,G", [(16, 5, 8, 2), (48, 7, 64, 2), (256, 32, 4, 1), (128, 1, 32, 1)])
+@pytest.mark.parametrize("V,W,H,G", [(16, 5, 8, 2), (48, 7, 64, 2), (256, 8, 4, 1), (128, 1, 32, 1)])
 def test_other_shapes(V, W, H, G):
     """Value dims, odd windows, 32 heads per group (the largest item), W = 1."""
     cfg = small(3, B=2, V=V, W=W, H=H, G=G, Hqk=H, n_dense=1)
     parity_run(cfg, 2 * W + 3)
+
+
+@pytest.mark.parametrize("cid", [1, 3, 4])
+def test_ring_reuse_moderate_batch(cid):
+    """Enough batch rows that every persistent decode CTA walks several units through
+    its stage ring (KDA's large dense items leave room for a one-stage ring)."""
+    cfg = small(cid, B=96)
+    parity_run(cfg, 18, rows=[0, 1, 47, 95])
 
 
 def test_single_row_batch():
