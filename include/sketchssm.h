@@ -188,6 +188,42 @@ sketchssm_status sketchssm_dense_decode(const sketchssm_plan *plan, int32_t pos,
                                         float *abuf, float *bbuf, const float *S, float *y,
                                         sketchssm_stream stream);
 
+/*
+ * Sketch decode whose scratch comes from a fixed static device array instead of the
+ * plan's buffer; the paper has no counterpart (it is a memory-ownership variant of
+ * sketchssm_decode, with the same arguments, layouts and results).
+ *
+ * For callers that must not allocate device memory at all once serving has started:
+ * an engine that has handed every free byte of HBM to its own state and KV pools, so
+ * that a cudaMalloc would fail or force its pool to give memory back, and code that
+ * cannot afford the device-wide synchronisation cudaMalloc / cudaFree may imply.
+ * This call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine): the coefficient / product rows live in one array of
+ * SKETCHSSM_STATIC_SCRATCH_BYTES per device, linked into the library.
+ *  - Limit: a plan whose sketch decode needs more than SKETCHSSM_STATIC_SCRATCH_BYTES
+ *    (Mamba-2: batch * qk_heads * round4(window + rank_cap) floats; GDN / KDA: batch
+ *    * the plan's coefficient floats per batch row) returns SKETCHSSM_ERR_INVALID_ARG
+ *    with the sizes in sketchssm_last_error(), before any tensor is looked at.
+ *  - Set-up: the first call on a device looks the array's address up there (with that
+ *    device current, which the plan check already requires); make that first call
+ *    before any stream capture.  Later calls only read the cached address.
+ *  - Sharing: every call on a device, from every plan and host thread, uses the same
+ *    array.  Calls whose kernels overlap on the GPU (different streams without an
+ *    ordering between them) race on it and give wrong results; calls in stream order
+ *    do not.
+ *  - Nothing in the array needs to start at zero: each call writes every scratch entry
+ *    it reads before reading it, so stale contents of an earlier call do not matter.
+ */
+#define SKETCHSSM_STATIC_SCRATCH_BYTES (8u << 20)
+
+sketchssm_status sketchssm_decode_static_scratch(const sketchssm_plan *plan, int32_t pos,
+                                                 const float *q, const float *k, const float *v,
+                                                 const float *a, const float *beta, float *kbuf,
+                                                 float *vbuf, float *abuf, float *bbuf,
+                                                 const float *Y, const float *omega,
+                                                 const float *S, float *y,
+                                                 sketchssm_stream stream);
+
 /* Static text of a status code. */
 const char *sketchssm_status_string(sketchssm_status status);
 

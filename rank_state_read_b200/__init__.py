@@ -15,6 +15,7 @@ from ._binding import (  # noqa: F401
     SketchSSMError,
     load,
     sketchssm_decode,
+    sketchssm_decode_static_scratch,
     sketchssm_dense_decode,
     sketchssm_flush,
     sketchssm_plan_create,

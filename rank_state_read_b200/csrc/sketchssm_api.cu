@@ -6,6 +6,7 @@
 
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "internal.cuh"
@@ -471,3 +472,84 @@ sketchssm_status sketchssm_dense_decode(const sketchssm_plan *p, int32_t pos, co
 }
 
 }  // extern "C"
+
+// ============================================================================ static scratch
+//
+// sketchssm_decode_static_scratch: the sketch decode with its scratch in a file-scope
+// static device array instead of the plan's cudaMalloc'd buffer.  It serves callers
+// that must not allocate device memory once serving has started (an engine whose HBM
+// is fully committed to its own state / KV pools, where a cudaMalloc would fail or
+// make the pool release memory, and code that cannot take the device-wide
+// synchronisation cudaMalloc / cudaFree may imply).  Nothing below allocates.
+//
+// The array is shared by every call on a device; calls that overlap on the GPU race
+// on it.  Nothing in it needs to start at zero: the products kernel writes every
+// entry the combine kernel reads before the combine reads it.
+
+static __device__ __align__(256) float g_static_scratch[SKETCHSSM_STATIC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+
+constexpr int STATIC_SCRATCH_DEVICES = 64;
+std::mutex g_static_mu;
+float *g_static_ptr[STATIC_SCRATCH_DEVICES];  // address of the array on each device
+
+// The array's address on device `dev`, which must be current.  Looked up by the first
+// call on that device, cached afterwards.
+sketchssm_status static_scratch(int dev, float **out)
+{
+    if (dev < 0 || dev >= STATIC_SCRATCH_DEVICES)
+        return fail(SKETCHSSM_ERR_UNSUPPORTED, "static scratch: device ordinal above 63");
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+        g_static_ptr[dev] = static_cast<float *>(p);
+    }
+    *out = g_static_ptr[dev];
+    return SKETCHSSM_OK;
+}
+
+// floats of scratch the sketch decode of plan p reads and writes
+size_t sketch_scratch_floats(const sketchssm_plan *p)
+{
+    const sketchssm_desc &d = p->d;
+    const size_t per_row = d.kind == SKETCHSSM_MAMBA2 ? (size_t)d.qk_heads * sk::dots_row(d.window, d.rank_cap)
+                                                      : (size_t)p->coef_row;
+    return per_row * (size_t)d.batch;
+}
+
+}  // namespace
+
+extern "C" sketchssm_status sketchssm_decode_static_scratch(const sketchssm_plan *p, int32_t pos, const float *q,
+                                                            const float *k, const float *v, const float *a,
+                                                            const float *beta, float *kbuf, float *vbuf,
+                                                            float *abuf, float *bbuf, const float *Y,
+                                                            const float *omega, const float *S, float *y,
+                                                            sketchssm_stream stream)
+{
+    g_last_error.clear();
+    sketchssm_status s = check_plan(p);
+    if (s != SKETCHSSM_OK) return s;
+    const size_t need = sketch_scratch_floats(p) * sizeof(float);
+    if (need > SKETCHSSM_STATIC_SCRATCH_BYTES)
+        return fail(SKETCHSSM_ERR_INVALID_ARG, "static scratch: this plan's decode needs " + std::to_string(need) +
+                                                   " bytes, the static array holds " +
+                                                   std::to_string(SKETCHSSM_STATIC_SCRATCH_BYTES) +
+                                                   " (use sketchssm_decode)");
+    if ((s = check_decode_common(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, y)) != SKETCHSSM_OK)
+        return s;
+    const sketchssm_desc &d = p->d;
+    const bool any_sketch = p->rtot > 0, any_dense = p->n_dense > 0;
+    CHECK_T(Y, any_sketch ? fbytes(d.batch, p->rtot, d.value_dim) : 0, "Y", !any_sketch);
+    CHECK_T(omega, any_sketch ? fbytes(d.groups, d.basis_rows, d.key_dim) : 0, "omega", !any_sketch);
+    CHECK_T(S, any_dense ? fbytes(d.batch, d.heads, d.key_dim, d.value_dim) : 0, "S", !any_dense);
+    float *scratch = nullptr;
+    if ((s = static_scratch(p->device, &scratch)) != SKETCHSSM_OK) return s;
+    sk::DecodeArgs A = decode_args(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, Y, omega, S, y, 0);
+    A.scratch = scratch;
+    cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch (static scratch)");
+    return SKETCHSSM_OK;
+}
