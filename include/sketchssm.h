@@ -110,8 +110,8 @@ typedef void *sketchssm_stream;
  * (rank + n per head) fit one shared-memory stage.  The plan owns those device
  * tables (freed by sketchssm_plan_destroy).  Synchronises `stream` once, so that
  * the host knows Rtot and the item counts.  *out is set only on success.
- * Source: the per-head "rank or a dense fallback" of the calibration stage
- * "allocate" (sketchssm PyPI page) and the group-shared basis of stage "basis".
+ * Source: the calibration stage "allocate" of the sketchssm PyPI page (each head
+ * gets a rank or falls back to dense) and its stage "basis" (one basis per group).
  */
 sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t *rank_host,
                                        sketchssm_stream stream, sketchssm_plan **out);
@@ -143,9 +143,9 @@ sketchssm_status sketchssm_plan_check(const sketchssm_plan *plan, sketchssm_stre
 sketchssm_status sketchssm_plan_destroy(sketchssm_plan *plan);
 
 /*
- * Flush (write-full step; paper abstract: "preserves full-state updates" and "reads
- * the full state once to precompute outputs for these basis vectors, storing them
- * in a compact sketch").  For every (b, h) apply buffer slots 0..n_tokens-1 in
+ * Flush (write-full step; paper abstract: updates always reach the full state, which
+ * is read only here, once, to compute the basis outputs kept as the sketch).  For
+ * every (b, h) apply buffer slots 0..n_tokens-1 in
  * order to S (in place), then write Y rows of every sketch head:
  *     Y[b][off[h] + m][:] = sum_k omega[g(h)][m][k] S[b][h][k][:],  m < rank[h].
  * n_tokens in [0, W]; with 0, S is left untouched and only Y is formed.

@@ -42,7 +42,7 @@ typedef struct {
 } oracle_dims;
 
 /* ------------------------------------------------------------------ layout
- * Packed sketch layout of one layer [PYPI "allocate"; ABS "compact sketch"]:
+ * Packed sketch layout of one layer [PYPI stage "allocate"; ABS, the sketch]:
  * off[h] = sum of the ranks of the sketch heads before h (dense heads own no rows),
  * off[H] = Rtot; rmax[g] = largest sketch rank in group g (0 if none).
  * Returns Rtot, or -1 if a rank is neither DENSE nor >= 1. */
@@ -68,13 +68,13 @@ static double a_scalar(const oracle_dims *d, const double *abuf, int64_t bh, int
 }
 
 /* ------------------------------------------------------------------ flush
- * Write-full step [ABS "preserves full-state updates"]: for every (b, h) apply the n
+ * Write-full step [ABS: every update reaches the full state]: for every (b, h) apply the n
  * buffered tokens in order, S <- M_i S + beta_i k_i v_i^T with
  *   Mamba-2: M_i = a_i I, beta_i = 1
  *   GDN:     M_i = a_i (I - beta_i k_i k_i^T)
  *   KDA:     M_i = diag(a_i) (I - beta_i k_i k_i^T)
  * then read the new state once to form the sketch of every sketch head
- * [ABS "reads the full state once to precompute outputs for these basis vectors"]:
+ * [ABS: the one read of the state, at the update, yields the basis outputs]:
  *   Y[off[h] + m][:] = sum_k omega[g][m][k] S[k][:]   for m < rank[h].
  * Dense heads keep no sketch. */
 void oracle_flush(const oracle_dims *d, const int32_t *rank, const int32_t *off, int64_t rtot,
@@ -143,7 +143,7 @@ void oracle_flush(const oracle_dims *d, const int32_t *rank, const int32_t *off,
  * seen by the flushed state S_f.
  *
  * State read: dense head (or dense_all) -> S_f^T q0 exactly [PYPI "dense fallback"];
- * sketch head [ABS "combines the sketch vectors with query-dependent coefficients"]:
+ * sketch head [ABS: sketch rows mixed with coefficients that depend on the query]:
  *   c_m = omega[g][m] . q0 (m < rank),  y_state = sum_m c_m Y[off + m][:].
  * y = y_state + y_rep. */
 void oracle_decode(const oracle_dims *d, const int32_t *rank, const int32_t *off, int64_t rtot,

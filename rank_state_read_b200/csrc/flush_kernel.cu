@@ -1,8 +1,9 @@
 // Flush: the write-full step (one launch every W decode steps).
 //
-// Paper abstract (SketchSSM): the method "preserves full-state updates", and "at
-// each state update ... reads the full state once to precompute outputs for these
-// basis vectors, storing them in a compact sketch".  For every (batch row, head):
+// SketchSSM (paper abstract): the state keeps receiving every update in full, and
+// the only time it is read is at a state update, where one pass over it computes the
+// outputs for the fixed basis vectors and stores them as the compact sketch.  For
+// every (batch row, head):
 //   1. apply the n buffered tokens in order, S <- M_i S + beta_i k_i v_i^T
 //      (Mamba-2 in closed form: S <- P S + sum_i w_i k_i v_i^T with
 //       P = prod_i a_i, w_i = prod_{j>i} a_j);
@@ -10,222 +11,492 @@
 //   3. for a sketch head, Y[off + m] = Omega_g[m] S for m < rank, from the S still
 //      held in registers, so S crosses HBM once each way.
 //
-// One CTA per (b, h, column slab of VS <= 128 columns); columns of S evolve
-// independently, so a slab is self-contained.  2 VS threads: thread (ks, c4) holds
-// the float4 column chunk c4 of the 16 consecutive state rows 16 ks .. 16 ks + 15,
-// and a warp covers 4 column chunks x 8 row slices, so every reduction over k (the
-// delta-rule erase term k^T S and the projection Omega S) is 3 xor-shuffle steps
-// inside the warp.  The state loads are issued first, straight into registers, and
-// fly while the CTA stages the buffered tokens in shared memory; keys and KDA decays
-// are staged with 4 floats of padding per 16 so that the float4 reads of the 8 row
-// slices fall on disjoint banks.  The basis rows are read through L1.
+// Work item: (b, h, column slab of VS columns); columns of S evolve independently,
+// so a slab is self-contained.  A persistent CTA walks a contiguous range of items
+// (consecutive heads of a batch row) with VS/16 compute warps and one producer warp.
+// Compute thread (ks, c4) holds the float4 column chunk c4 of the 16 state rows
+// 4 ks + 32 q + e (q, e < 4); a warp covers 4 column chunks x 8 row slices, so every
+// reduction over k (the delta-rule erase term k^T S and the projection Omega S) stays
+// inside the warp, and the float4 reads of keys, decays and basis rows by the 8 row
+// slices are 128 consecutive bytes (no bank conflict, no padding).
+//
+// Data movement is TMA bulk copies (cp.async.bulk, completion counted on an mbarrier),
+// which keep far more bytes in flight per SM than register loads.  The producer warp
+// requests, one item ahead:
+//   - the item's state slab into one shared buffer, as 32 chunks of 4 rows, each
+//     chunk padded by 4 floats so that the 8 row slices' float4 reads fall on
+//     disjoint banks;
+//   - the buffered keys, values and KDA decays into one of two token buffers;
+//   - when the head group changes, the basis rows 0 .. rmax_g - 1 of the new group,
+//     which stay resident while the group lasts.
+// Handshake: `full` completes when an item's copies have landed; every compute warp
+// arrives on `empty` once it has the slab in registers (by then it is also done with
+// the previous item), which frees the slab buffer, the other token buffer and the
+// basis rows for the producer.  No CTA-wide barrier in the loop.  State and sketch rows
+// are written straight from registers; the per-token scalars a_i, beta_i are loaded
+// one item ahead into the lanes < n and broadcast by shuffles.
 #include "device_util.cuh"
 #include "internal.cuh"
+#include "ptx_util.cuh"
 
 namespace sk {
 namespace {
 
-constexpr int RPT = KDIM / 8;          // state rows per thread (16)
-constexpr int KPAD = KDIM + KDIM / 4;  // padded key row: 4 pad floats per 16
+constexpr int QROWS = KDIM / 32;  // row quads per thread (4): rows 4 ks + 32 q + e
+constexpr int FLUSH_MAXT = 192;   // up to 5 compute warps (VS <= 80) + the producer
 
-__device__ __forceinline__ int kpad(int k) { return k + (k >> 4) * 4; }
+struct FlushCarve {
+    size_t bar, S, T, O, total;          // byte offsets in shared memory
+    size_t tkeys, tv, ta, tfloats;       // float offsets within one token buffer
+};
 
-__host__ __device__ inline size_t flush_smem_floats(int kind, int VS, int W)
+__host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
+
+__host__ __device__ inline FlushCarve flush_carve(int kind, int VS, int W, int rcap)
 {
-    return (size_t)W * KPAD + (size_t)W * VS + 2 * (size_t)W + (kind == SKETCHSSM_KDA ? (size_t)W * KPAD : 0);
+    FlushCarve c;
+    c.tkeys = 0;
+    c.tv = (size_t)W * KDIM;
+    c.ta = c.tv + (size_t)W * VS;
+    c.tfloats = c.ta + (kind == SKETCHSSM_KDA ? (size_t)W * KDIM : 0);
+    size_t o = 0;
+    c.bar = o;  // full, empty, omega barriers and the abort flag
+    o = align128(o + 4 * sizeof(uint64_t));
+    c.S = o;
+    o = align128(o + sizeof(float) * 32 * (size_t)(4 * VS + 4));
+    c.T = o;
+    o = align128(o + 2 * sizeof(float) * c.tfloats);
+    c.O = o;
+    o = align128(o + sizeof(float) * (size_t)rcap * KDIM);
+    c.total = o;
+    return c;
 }
 
-template <int KIND, int MAXT, int MINB>
-__global__ void __launch_bounds__(MAXT, MINB)
+// (b, h, slab) of consecutive items, advanced without divisions
+struct Cursor {
+    int b, h, slab, r;
+    __device__ void init(const FlushArgs &A, long long item, int nslab)
+    {
+        const long long bh = item / nslab;
+        slab = (int)(item - bh * nslab);
+        b = (int)(bh / A.H);
+        h = (int)(bh - (long long)b * A.H);
+        r = __ldg(A.rank + h);
+    }
+    __device__ void next(const FlushArgs &A, int nslab)
+    {
+        if (++slab == nslab) {
+            slab = 0;
+            if (++h == A.H) {
+                h = 0;
+                ++b;
+            }
+            r = __ldg(A.rank + h);
+        }
+    }
+    __device__ long long bh(const FlushArgs &A) const { return (long long)b * A.H + h; }
+};
+
+// Wait for phase `parity` of `bar`, giving up after `limit` cycles or when another
+// warp of the CTA has given up (abort flag set).
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, long long limit,
+                                              const volatile int *abort)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort || clock64() - t0 > limit) return false;
+    }
+    return true;
+}
+
+// The producer warp requests an item's state slab and (n > 0) its buffered tokens,
+// all counted on `bar`.  An item with nothing to do (n = 0 and a dense head) arrives
+// on the barrier with no bytes.
+template <int KIND>
+__device__ __forceinline__ void issue_item(const FlushArgs &A, const Cursor &it, int nslab, float *Sbuf,
+                                           float *T, const FlushCarve &cv, uint64_t *bar, int lane)
+{
+    const int V = A.V, VS = A.VS, W = A.W, n = A.n;
+    const bool needed = n > 0 || it.r > 0;
+    if (lane == 0) {
+        uint32_t bytes = 0;
+        if (needed) {
+            bytes = (uint32_t)(KDIM * VS * 4);
+            if (n > 0) {
+                bytes += (uint32_t)(n * KDIM * 4 + n * VS * 4);
+                if (KIND == SKETCHSSM_KDA) bytes += (uint32_t)(n * KDIM * 4);
+            }
+        }
+        mbar_arrive_expect_tx(bar, bytes);
+    }
+    __syncwarp();
+    if (!needed) return;
+    const long long bh = it.bh(A);
+    const float *Sg = A.S + bh * KDIM * V + (long long)it.slab * VS;
+    float *dst = Sbuf + (size_t)lane * (4 * VS + 4);
+    if (nslab == 1) {  // 4 state rows are 4 V contiguous floats
+        bulk_copy_g2s(dst, Sg + (long long)lane * 4 * V, (uint32_t)(16 * VS), bar);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            bulk_copy_g2s(dst + e * VS, Sg + (long long)(lane * 4 + e) * V, (uint32_t)(4 * VS), bar);
+    }
+    if (n > 0) {
+        const int qk = it.h / A.hpq;
+        if (lane == 0)
+            bulk_copy_g2s(T + cv.tkeys, A.kbuf + ((long long)it.b * A.Hqk + qk) * W * KDIM,
+                          (uint32_t)(n * KDIM * 4), bar);
+        if (KIND == SKETCHSSM_KDA && lane == 1)
+            bulk_copy_g2s(T + cv.ta, A.abuf + bh * W * KDIM, (uint32_t)(n * KDIM * 4), bar);
+        const float *vg = A.vbuf + bh * W * V + (long long)it.slab * VS;
+        if (nslab == 1) {
+            if (lane == 2) bulk_copy_g2s(T + cv.tv, vg, (uint32_t)(n * V * 4), bar);
+        } else {
+            for (int i = lane; i < n; i += 32)
+                bulk_copy_g2s(T + cv.tv + (size_t)i * VS, vg + (long long)i * V, (uint32_t)(VS * 4), bar);
+        }
+    }
+}
+
+// s += c * x, for the 4 rows of a row quad held as s[0..3] and c = (c.x .. c.w)
+__device__ __forceinline__ void quad_rank1(float4 *s, float4 c, float4 x)
+{
+    fma4(s[0], c.x, x);
+    fma4(s[1], c.y, x);
+    fma4(s[2], c.z, x);
+    fma4(s[3], c.w, x);
+}
+
+// acc += sum_e c_e s[e] over a row quad
+__device__ __forceinline__ void quad_dot(float4 &acc, float4 c, const float4 *s)
+{
+    fma4(acc, c.x, s[0]);
+    fma4(acc, c.y, s[1]);
+    fma4(acc, c.z, s[2]);
+    fma4(acc, c.w, s[3]);
+}
+
+__device__ __forceinline__ float4 add4(float4 a, float4 b)
+{
+    return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+__device__ __forceinline__ float4 shfl_xor4(float4 v, int m)
+{
+    return make_float4(__shfl_xor_sync(0xffffffffu, v.x, m), __shfl_xor_sync(0xffffffffu, v.y, m),
+                       __shfl_xor_sync(0xffffffffu, v.z, m), __shfl_xor_sync(0xffffffffu, v.w, m));
+}
+
+// One step of a reduce-scatter between lanes that differ in bit `m`: the lane with
+// the bit clear keeps lo (adds the partner's lo), the other keeps hi.
+__device__ __forceinline__ float4 rs_step(float4 lo, float4 hi, bool upper, int m)
+{
+    const float4 keep = upper ? hi : lo, send = upper ? lo : hi;
+    return add4(keep, shfl_xor4(send, m));
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(FLUSH_MAXT, 2)
 flush_kernel(const FlushArgs A)
 {
-    extern __shared__ __align__(16) float fsm[];
-    const int H = A.H, V = A.V, W = A.W, n = A.n, VS = A.VS;
+    extern __shared__ __align__(128) unsigned char fsm_raw[];
+    const int V = A.V, W = A.W, n = A.n, VS = A.VS;
     const int nslab = V / VS;
-    const long long item = blockIdx.x;
-    const long long bh = item / nslab;
-    const int slab = (int)(item - bh * nslab);
-    const int b = (int)(bh / H), h = (int)(bh - (long long)b * H);
-    const int r = __ldg(A.rank + h);
-    if (n == 0 && r <= 0) return;  // nothing to apply, nothing to project
+    const int ncw = VS / 16;  // compute warps
+    const FlushCarve cv = flush_carve(KIND, VS, W, A.rcap);
+    uint64_t *full = reinterpret_cast<uint64_t *>(fsm_raw + cv.bar);
+    uint64_t *empty = full + 1;
+    uint64_t *obar = full + 2;
+    volatile int *abort = reinterpret_cast<volatile int *>(full + 3);
+    float *Sbuf = reinterpret_cast<float *>(fsm_raw + cv.S);
+    float *Tb = reinterpret_cast<float *>(fsm_raw + cv.T);
+    float *Obuf = reinterpret_cast<float *>(fsm_raw + cv.O);
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, T = blockDim.x;
-    const int ks = lane & 7;
-    const int c4 = warp * 4 + (lane >> 3);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // 1. the state slab, straight into registers
-    float *Sg = A.S + (bh * KDIM + ks * RPT) * V + slab * VS + c4 * 4;
-    float4 s[RPT];
-#pragma unroll
-    for (int j = 0; j < RPT; ++j) s[j] = ldg4(Sg + (long long)j * V);
+    const long long items = (long long)A.B * A.H * nslab;
+    const long long first = items * blockIdx.x / gridDim.x;
+    const long long last = items * (blockIdx.x + 1) / gridDim.x;
+    if (first >= last) return;
+    const int cnt = (int)(last - first);
 
-    // 2. buffered tokens into shared memory
-    float *kt = fsm;                 // [W][KPAD] keys
-    float *vt = kt + W * KPAD;       // [W][VS]   values of the slab
-    float *sc = vt + W * VS;         // [2W]      a_i (or alpha_i), beta_i
-    float *av = sc + 2 * W;          // [W][KPAD] KDA decays
-    if (n > 0) {
-        const int qk = h / A.hpq;
-        const float *kg = A.kbuf + ((long long)b * A.Hqk + qk) * W * KDIM;
-        for (int x = tid; x < n * (KDIM / 4); x += T) {
-            const int i = x / (KDIM / 4), c = x - i * (KDIM / 4);
-            st4(kt + i * KPAD + kpad(c * 4), ldg4(kg + (long long)i * KDIM + c * 4));
-            if (KIND == SKETCHSSM_KDA)
-                st4(av + i * KPAD + kpad(c * 4), ldg4(A.abuf + (bh * W + i) * KDIM + c * 4));
-        }
-        const int VS4 = VS / 4;
-        for (int x = tid; x < n * VS4; x += T) {
-            const int i = x / VS4, c = x - i * VS4;
-            st4(vt + i * VS + c * 4, ldg4(A.vbuf + (bh * W + i) * V + slab * VS + c * 4));
-        }
-        if (tid < n) {
-            if (KIND != SKETCHSSM_KDA) sc[tid] = __ldg(A.abuf + bh * W + tid);
-            if (KIND != SKETCHSSM_MAMBA2) sc[W + tid] = __ldg(A.bbuf + bh * W + tid);
-        }
+    if (tid == 0) {
+        mbar_init(full, 1);
+        mbar_init(empty, ncw);
+        mbar_init(obar, 1);
+        *abort = 0;
+        mbar_fence_init();
     }
     __syncthreads();
 
-    // 3. the update
-    const float *ktr = kt + ks * 20;  // = kpad(16 ks)
-    if (KIND == SKETCHSSM_MAMBA2) {
+    Cursor cur;
+    cur.init(A, first, nslab);
+    int g_loaded = -1;
+    // does this item start a new head group with sketch rows? (tracked alike by all warps)
+    auto new_group = [&](const Cursor &c) {
+        if (c.r <= 0) return false;
+        const int g = c.h / A.Hg;
+        if (g == g_loaded) return false;
+        g_loaded = g;
+        return true;
+    };
+
+    if (warp == ncw) {
+        // ------------------------------------------------------------ producer
+        uint32_t last_full = 0, last_o = 0;
+        int issued_o = 0;
+        auto issue_omega = [&](const Cursor &c) {
+            if (lane == 0) {
+                const int g = c.h / A.Hg;
+                const uint32_t bytes = (uint32_t)(__ldg(A.rmax + g) * KDIM * 4);
+                mbar_arrive_expect_tx(obar, bytes);
+                bulk_copy_g2s(Obuf, A.omega + (long long)g * A.Rb * KDIM, bytes, obar);
+            }
+            last_o = (uint32_t)(issued_o & 1);
+            ++issued_o;
+        };
+        bool pend_o = new_group(cur);
+        issue_item<KIND>(A, cur, nslab, Sbuf, Tb, cv, full, lane);
+        if (pend_o) issue_omega(cur);
+        pend_o = false;
+        bool ok = true;
+        for (int j = 1; j <= cnt; ++j) {
+            // every compute warp holds item j-1's slab and is done with item j-2
+            ok = wait_or_abort(empty, (uint32_t)((j - 1) & 1), A.wait_limit, abort);
+            if (!ok) break;
+            if (pend_o) issue_omega(cur);  // item j-1's new basis rows
+            pend_o = false;
+            if (j == cnt) break;
+            cur.next(A, nslab);
+            pend_o = new_group(cur) && j > 0;
+            issue_item<KIND>(A, cur, nslab, Sbuf, Tb + (size_t)(j & 1) * cv.tfloats, cv, full, lane);
+            last_full = (uint32_t)(j & 1);
+        }
+        if (!ok) {
+            if (lane == 0) {
+                *abort = 1;
+                atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
+            }
+            // copies still in flight land before the CTA's shared memory is released
+            mbar_wait_bounded(full, last_full, A.wait_limit);
+            if (issued_o > 0) mbar_wait_bounded(obar, last_o, A.wait_limit);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- compute warps
+    const int ks = lane & 7;
+    const int c4 = warp * 4 + (lane >> 3);
+    // per-token scalars of the current item in lanes < n
+    float a_l = 1.f, b_l = 0.f;
+    auto load_scalars = [&](const Cursor &c, float &a, float &bv) {
+        a = 1.f;
+        bv = 0.f;
+        if (lane < n) {
+            const long long o = c.bh(A) * W + lane;
+            if (KIND != SKETCHSSM_KDA) a = __ldg(A.abuf + o);
+            if (KIND != SKETCHSSM_MAMBA2) bv = __ldg(A.bbuf + o);
+        }
+    };
+    load_scalars(cur, a_l, b_l);
+    uint32_t o_phase = 0;
+
+    for (int j = 0; j < cnt; ++j) {
+        const float *T = Tb + (size_t)(j & 1) * cv.tfloats;
+        const int r = cur.r;
+        const bool need_o = new_group(cur);
+
+        if (!wait_or_abort(full, (uint32_t)(j & 1), A.wait_limit, abort)) {
+            if (lane == 0) {
+                *abort = 1;
+                atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
+            }
+            return;
+        }
+        float4 s[16];
+        {
+            const float *sb = Sbuf + (size_t)ks * (4 * VS + 4) + c4 * 4;
+#pragma unroll
+            for (int q = 0; q < QROWS; ++q)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) s[4 * q + e] = lds4(sb + (size_t)q * 8 * (4 * VS + 4) + e * VS);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty);
+
+        // the next item's scalars, one item ahead
+        Cursor nxt = cur;
+        float a_n = 1.f, b_n = 0.f;
+        if (j + 1 < cnt) {
+            nxt.next(A, nslab);
+            load_scalars(nxt, a_n, b_n);
+        }
+
+        // the update
+        const float *kt = T + cv.tkeys + 4 * ks;
+        const float *vt = T + cv.tv + c4 * 4;
+        if (KIND == SKETCHSSM_MAMBA2) {
+            if (n > 0) {
+                float P = a_l;  // prod of a_i over the lanes (lanes >= n hold 1)
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) P *= __shfl_xor_sync(0xffffffffu, P, o);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    s[q].x *= P; s[q].y *= P; s[q].z *= P; s[q].w *= P;
+                }
+                float w = 1.f;  // w_i = prod_{j>i} a_j, newest token first
+                for (int i = n - 1; i >= 0; --i) {
+                    float4 vv = lds4(vt + i * VS);
+                    vv.x *= w; vv.y *= w; vv.z *= w; vv.w *= w;
+                    const float *ki = kt + i * KDIM;
+#pragma unroll
+                    for (int q = 0; q < QROWS; ++q) quad_rank1(s + 4 * q, lds4(ki + q * 32), vv);
+                    w *= __shfl_sync(0xffffffffu, a_l, i);
+                }
+            }
+        } else {
+            const float *at = T + cv.ta + 4 * ks;
+            for (int i = 0; i < n; ++i) {
+                const float *ki = kt + i * KDIM;
+                float4 kq[QROWS];
+#pragma unroll
+                for (int q = 0; q < QROWS; ++q) kq[q] = lds4(ki + q * 32);
+                float4 d0 = zero4(), d1 = zero4();
+                quad_dot(d0, kq[0], s + 0);
+                quad_dot(d1, kq[1], s + 4);
+                quad_dot(d0, kq[2], s + 8);
+                quad_dot(d1, kq[3], s + 12);
+                const float4 d = sum8_xor(add4(d0, d1));  // d = S^T k_i for this column chunk
+                const float4 vv = lds4(vt + i * VS);
+                const float bi = __shfl_sync(0xffffffffu, b_l, i);
+                if (KIND == SKETCHSSM_GDN) {
+                    // a (S - beta k d) + beta k v = a S + k * beta (v - a d)
+                    const float ai = __shfl_sync(0xffffffffu, a_l, i);
+                    const float4 u = make_float4(bi * fmaf(-ai, d.x, vv.x), bi * fmaf(-ai, d.y, vv.y),
+                                                 bi * fmaf(-ai, d.z, vv.z), bi * fmaf(-ai, d.w, vv.w));
+#pragma unroll
+                    for (int q = 0; q < QROWS; ++q) {
+                        const float kk[4] = {kq[q].x, kq[q].y, kq[q].z, kq[q].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float4 &t = s[4 * q + e];
+                            t.x = fmaf(ai, t.x, kk[e] * u.x);
+                            t.y = fmaf(ai, t.y, kk[e] * u.y);
+                            t.z = fmaf(ai, t.z, kk[e] * u.z);
+                            t.w = fmaf(ai, t.w, kk[e] * u.w);
+                        }
+                    }
+                } else {
+                    // a_k (S - beta k_k d) + beta k_k v = a_k S + beta k_k (v - a_k d)
+                    const float *ai = at + i * KDIM;
+#pragma unroll
+                    for (int q = 0; q < QROWS; ++q) {
+                        const float4 a4 = lds4(ai + q * 32);
+                        const float kk[4] = {kq[q].x, kq[q].y, kq[q].z, kq[q].w};
+                        const float aq[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float4 &t = s[4 * q + e];
+                            const float ak = aq[e], kb = bi * kk[e];
+                            t.x = fmaf(ak, t.x, kb * fmaf(-ak, d.x, vv.x));
+                            t.y = fmaf(ak, t.y, kb * fmaf(-ak, d.y, vv.y));
+                            t.z = fmaf(ak, t.z, kb * fmaf(-ak, d.z, vv.z));
+                            t.w = fmaf(ak, t.w, kb * fmaf(-ak, d.w, vv.w));
+                        }
+                    }
+                }
+            }
+        }
+        const long long bh = cur.bh(A);
         if (n > 0) {
-            float P = 1.f;
-            for (int i = 0; i < n; ++i) P *= sc[i];
+            float *Sg = A.S + (bh * KDIM + 4 * ks) * V + (long long)cur.slab * VS + c4 * 4;
 #pragma unroll
-            for (int j = 0; j < RPT; ++j) {
-                s[j].x *= P; s[j].y *= P; s[j].z *= P; s[j].w *= P;
-            }
-            float w = 1.f;  // w_i = prod_{j>i} a_j, newest token first
-            for (int i = n - 1; i >= 0; --i) {
-                float4 vv = lds4(vt + i * VS + c4 * 4);
-                vv.x *= w; vv.y *= w; vv.z *= w; vv.w *= w;
-                const float *ki = ktr + i * KPAD;
+            for (int q = 0; q < QROWS; ++q)
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 kk = lds4(ki + q * 4);
-                    fma4(s[4 * q + 0], kk.x, vv);
-                    fma4(s[4 * q + 1], kk.y, vv);
-                    fma4(s[4 * q + 2], kk.z, vv);
-                    fma4(s[4 * q + 3], kk.w, vv);
-                }
-                w *= sc[i];
-            }
+                for (int e = 0; e < 4; ++e) st4(Sg + (long long)(32 * q + e) * V, s[4 * q + e]);
         }
-    } else {
-        const float *avr = av + ks * 20;
-        for (int i = 0; i < n; ++i) {
-            const float *ki = ktr + i * KPAD;
-            float4 d = zero4();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 kk = lds4(ki + q * 4);
-                fma4(d, kk.x, s[4 * q + 0]);
-                fma4(d, kk.y, s[4 * q + 1]);
-                fma4(d, kk.z, s[4 * q + 2]);
-                fma4(d, kk.w, s[4 * q + 3]);
-            }
-            d = sum8_xor(d);  // d = S^T k_i for this column chunk
-            const float4 vv = lds4(vt + i * VS + c4 * 4);
-            const float bi = sc[W + i];
-            if (KIND == SKETCHSSM_GDN) {
-                // a (S - beta k d) + beta k v = a S + k * beta (v - a d)
-                const float ai = sc[i];
-                const float4 u = make_float4(bi * fmaf(-ai, d.x, vv.x), bi * fmaf(-ai, d.y, vv.y),
-                                             bi * fmaf(-ai, d.z, vv.z), bi * fmaf(-ai, d.w, vv.w));
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 kk = lds4(ki + q * 4);
-                    const float kq[4] = {kk.x, kk.y, kk.z, kk.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float4 &t = s[4 * q + e];
-                        t.x = fmaf(ai, t.x, kq[e] * u.x);
-                        t.y = fmaf(ai, t.y, kq[e] * u.y);
-                        t.z = fmaf(ai, t.z, kq[e] * u.z);
-                        t.w = fmaf(ai, t.w, kq[e] * u.w);
-                    }
-                }
-            } else {
-                // a_k (S - beta k_k d) + beta k_k v = a_k S + beta k_k (v - a_k d)
-                const float *ai = avr + i * KPAD;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 kk = lds4(ki + q * 4);
-                    const float4 a4 = lds4(ai + q * 4);
-                    const float kq[4] = {kk.x, kk.y, kk.z, kk.w};
-                    const float aq[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float4 &t = s[4 * q + e];
-                        const float ak = aq[e], kb = bi * kq[e];
-                        t.x = fmaf(ak, t.x, kb * fmaf(-ak, d.x, vv.x));
-                        t.y = fmaf(ak, t.y, kb * fmaf(-ak, d.y, vv.y));
-                        t.z = fmaf(ak, t.z, kb * fmaf(-ak, d.z, vv.z));
-                        t.w = fmaf(ak, t.w, kb * fmaf(-ak, d.w, vv.w));
-                    }
-                }
-            }
-        }
-    }
-    if (n > 0) {
-#pragma unroll
-        for (int j = 0; j < RPT; ++j) st4(Sg + (long long)j * V, s[j]);
-    }
 
-    // 4. the sketch rows of this slab, from registers
-    if (r > 0) {
-        float *Yh = A.Y + ((long long)b * A.rtot + __ldg(A.off + h)) * V + slab * VS + c4 * 4;
-        const float *og = A.omega + ((long long)(h / A.Hg) * A.Rb) * KDIM + ks * RPT;
-        for (int m = 0; m < r; ++m) {
-            const float *o = og + (long long)m * KDIM;
-            float4 p = zero4();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 om = ldg4(o + q * 4);
-                fma4(p, om.x, s[4 * q + 0]);
-                fma4(p, om.y, s[4 * q + 1]);
-                fma4(p, om.z, s[4 * q + 2]);
-                fma4(p, om.w, s[4 * q + 3]);
+        // the sketch rows of this slab: 8 rows at a time, reduced over the 8 row slices
+        // by a reduce-scatter that leaves row m0 + ks in lane ks
+        if (r > 0) {
+            if (need_o) {
+                if (!wait_or_abort(obar, o_phase, A.wait_limit, abort)) {
+                    if (lane == 0) {
+                        *abort = 1;
+                        atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
+                    }
+                    return;
+                }
+                o_phase ^= 1u;
             }
-            p = sum8_xor(p);
-            if (ks == (m & 7)) st4(Yh + (long long)m * V, p);
+            float *Yh = A.Y + ((long long)cur.b * A.rtot + __ldg(A.off + cur.h)) * V + (long long)cur.slab * VS +
+                        c4 * 4;
+            const float *om = Obuf + 4 * ks;
+            const bool u2 = ks & 4, u1 = ks & 2, u0 = ks & 1;
+            for (int m0 = 0; m0 < r; m0 += 8) {
+                float4 p[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    float4 x0 = zero4(), x1 = zero4();
+                    if (m0 + u < r) {
+                        const float *o = om + (m0 + u) * KDIM;
+                        quad_dot(x0, lds4(o), s + 0);
+                        quad_dot(x1, lds4(o + 32), s + 4);
+                        quad_dot(x0, lds4(o + 64), s + 8);
+                        quad_dot(x1, lds4(o + 96), s + 12);
+                    }
+                    p[u] = add4(x0, x1);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) p[u] = rs_step(p[u], p[u + 4], u2, 4);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) p[u] = rs_step(p[u], p[u + 2], u1, 2);
+                p[0] = rs_step(p[0], p[1], u0, 1);
+                if (m0 + ks < r) st4(Yh + (long long)(m0 + ks) * V, p[0]);
+            }
         }
+        cur = nxt;
+        a_l = a_n;
+        b_l = b_n;
     }
-}
-
-template <int KIND, int MAXT, int MINB>
-cudaError_t launch_cfg(const FlushArgs &a, cudaStream_t stream)
-{
-    const size_t smem = flush_smem_floats(KIND, a.VS, a.W) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(flush_kernel<KIND, MAXT, MINB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const long long blocks = (long long)a.B * a.H * (a.V / a.VS);
-    flush_kernel<KIND, MAXT, MINB><<<(unsigned)blocks, 2 * a.VS, smem, stream>>>(a);
-    return cudaGetLastError();
 }
 
 template <int KIND>
 cudaError_t launch_kind(const FlushArgs &a, cudaStream_t stream)
 {
-    // slabs of up to 80 columns run 160-thread CTAs, four per SM; wider slabs 256
-    if (2 * a.VS <= 160) return launch_cfg<KIND, 160, 4>(a, stream);
-    return launch_cfg<KIND, 256, 2>(a, stream);
+    const FlushCarve cv = flush_carve(KIND, a.VS, a.W, a.rcap);
+    const int threads = 32 * (a.VS / 16 + 1);
+    auto kern = flush_kernel<KIND>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cv.total);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, cv.total)) != cudaSuccess)
+        return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const long long items = (long long)a.B * a.H * (a.V / a.VS);
+    long long grid = (long long)per_sm * sms;
+    if (grid > items) grid = items;
+    kern<<<(unsigned)grid, threads, cv.total, stream>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 int flush_slab(int V)
 {
-    if (V <= 128) return V;
-    for (int vs = 128; vs >= 16; vs -= 16)
+    // up to 80 columns in one slab; wider states in slabs of at most 64 columns, so
+    // that the slab buffer, two token buffers and the basis rows fit shared memory
+    if (V <= 80) return V;
+    for (int vs = 64; vs >= 16; vs -= 16)
         if (V % vs == 0) return vs;
     return 16;
 }
 
-size_t flush_smem_bytes(int kind, int V, int W)
+size_t flush_smem_bytes(int kind, int V, int W, int rcap)
 {
-    return flush_smem_floats(kind, flush_slab(V), W) * sizeof(float);
+    return flush_carve(kind, flush_slab(V), W, rcap).total;
 }
 
 cudaError_t launch_flush(const FlushArgs &a, cudaStream_t stream)

@@ -17,6 +17,7 @@ constexpr int MAX_V = 256;       // value dim
 
 // bits of the plan's device status word
 constexpr int SK_STATUS_DECODE_TIMEOUT = 1;
+constexpr int SK_STATUS_FLUSH_TIMEOUT = 2;
 
 // default bound of a kernel's wait on its own bulk copies (clock cycles, ~1 s)
 constexpr long long DEFAULT_WAIT_CYCLES = 2000000000LL;
@@ -55,7 +56,11 @@ struct DecodeArgs {
 struct FlushArgs {
     int kind, B, H, Hqk, V, W, G, Rb, cap, n;
     int Hg, hpq;
-    int VS;  // column slab of one work item
+    int VS;    // column slab of one work item
+    int rcap;  // the largest sketch rank of the plan (0 if none): basis rows staged per CTA
+    const int *rmax;          // [G] largest sketch rank per group
+    int *status;              // plan status word (timeouts)
+    long long wait_limit;     // clock cycles of a bounded wait
     int64_t rtot;
     const int *rank, *off;
     float *S;
@@ -76,7 +81,7 @@ size_t decode_smem_bytes(const DecodeArgs &a);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
 int flush_slab(int V);
-size_t flush_smem_bytes(int kind, int V, int W);
+size_t flush_smem_bytes(int kind, int V, int W, int rcap);
 cudaError_t launch_flush(const FlushArgs &a, cudaStream_t stream);
 
 // Layout kernel: off[H+1], rmax[G], coff[H], per-n work lists work[(n-1)(H+G) ...];

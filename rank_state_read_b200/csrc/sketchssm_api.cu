@@ -362,6 +362,8 @@ sketchssm_status sketchssm_plan_check(const sketchssm_plan *p, sketchssm_stream 
     if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream");
     if (flags & sk::SK_STATUS_DECODE_TIMEOUT)
         return fail(SKETCHSSM_ERR_TIMEOUT, "a decode CTA gave up waiting for its bulk copies; its outputs are incomplete");
+    if (flags & sk::SK_STATUS_FLUSH_TIMEOUT)
+        return fail(SKETCHSSM_ERR_TIMEOUT, "a flush CTA gave up waiting for its bulk copies; S and Y are incomplete");
     return SKETCHSSM_OK;
 }
 
@@ -417,6 +419,11 @@ sketchssm_status sketchssm_flush(const sketchssm_plan *p, float *S, const float 
     A.Hg = p->Hg;
     A.hpq = p->hpq;
     A.VS = sk::flush_slab(d.value_dim);
+    A.rcap = 0;
+    for (int r : p->h_rmax) A.rcap = r > A.rcap ? r : A.rcap;
+    A.rmax = p->d_rmax;
+    A.status = p->d_status;
+    A.wait_limit = p->wait_limit;
     A.rtot = p->rtot;
     A.rank = p->d_rank;
     A.off = p->d_off;
