@@ -1,8 +1,8 @@
 // Sketch decode and dense-read decode: two launches per decode step.
 //
-// Paper abstract (SketchSSM, newx.sg / mlsanity pages): a decode step "combines the
-// sketch vectors with query-dependent coefficients to reconstruct the output
-// without a full-state read"; the buffered keys and values since the last state
+// Paper abstract (SketchSSM, newx.sg / mlsanity pages): a decode step rebuilds the
+// output from the sketch rows weighted by coefficients computed from the query, and
+// never reads the full state; the keys and values buffered since the last state
 // update (ReplaySSM) are replayed exactly.  A head with a dense fallback (PyPI page,
 // stage "allocate") reads the full state instead; the dense-read baseline does that
 // for every head.

@@ -72,9 +72,10 @@ __host__ __device__ inline FlushCarve flush_carve(int kind, int VS, int W, int r
     return c;
 }
 
-// (b, h, slab) of consecutive items, advanced without divisions
+// (b, h, slab) of consecutive items, advanced without divisions; the head's rank and
+// sketch-row offset are loaded when the cursor moves (one item before they are used)
 struct Cursor {
-    int b, h, slab, r;
+    int b, h, slab, r, off;
     __device__ void init(const FlushArgs &A, long long item, int nslab)
     {
         const long long bh = item / nslab;
@@ -82,6 +83,7 @@ struct Cursor {
         b = (int)(bh / A.H);
         h = (int)(bh - (long long)b * A.H);
         r = __ldg(A.rank + h);
+        off = __ldg(A.off + h);
     }
     __device__ void next(const FlushArgs &A, int nslab)
     {
@@ -92,6 +94,7 @@ struct Cursor {
                 ++b;
             }
             r = __ldg(A.rank + h);
+            off = __ldg(A.off + h);
         }
     }
     __device__ long long bh(const FlushArgs &A) const { return (long long)b * A.H + h; }
@@ -244,18 +247,18 @@ flush_kernel(const FlushArgs A)
     if (warp == ncw) {
         // ------------------------------------------------------------ producer
         uint32_t last_full = 0, last_o = 0;
-        int issued_o = 0;
+        int issued_o = 0, o_rows = 0;
         auto issue_omega = [&](const Cursor &c) {
             if (lane == 0) {
-                const int g = c.h / A.Hg;
-                const uint32_t bytes = (uint32_t)(__ldg(A.rmax + g) * KDIM * 4);
+                const uint32_t bytes = (uint32_t)(o_rows * KDIM * 4);
                 mbar_arrive_expect_tx(obar, bytes);
-                bulk_copy_g2s(Obuf, A.omega + (long long)g * A.Rb * KDIM, bytes, obar);
+                bulk_copy_g2s(Obuf, A.omega + (long long)(c.h / A.Hg) * A.Rb * KDIM, bytes, obar);
             }
             last_o = (uint32_t)(issued_o & 1);
             ++issued_o;
         };
         bool pend_o = new_group(cur);
+        if (pend_o) o_rows = __ldg(A.rmax + cur.h / A.Hg);
         issue_item<KIND>(A, cur, nslab, Sbuf, Tb, cv, full, lane);
         if (pend_o) issue_omega(cur);
         pend_o = false;
@@ -268,7 +271,8 @@ flush_kernel(const FlushArgs A)
             pend_o = false;
             if (j == cnt) break;
             cur.next(A, nslab);
-            pend_o = new_group(cur) && j > 0;
+            pend_o = new_group(cur);
+            if (pend_o) o_rows = __ldg(A.rmax + cur.h / A.Hg);  // used one iteration later
             issue_item<KIND>(A, cur, nslab, Sbuf, Tb + (size_t)(j & 1) * cv.tfloats, cv, full, lane);
             last_full = (uint32_t)(j & 1);
         }
@@ -344,14 +348,28 @@ flush_kernel(const FlushArgs A)
                 for (int q = 0; q < 16; ++q) {
                     s[q].x *= P; s[q].y *= P; s[q].z *= P; s[q].w *= P;
                 }
-                float w = 1.f;  // w_i = prod_{j>i} a_j, newest token first
-                for (int i = n - 1; i >= 0; --i) {
-                    float4 vv = lds4(vt + i * VS);
-                    vv.x *= w; vv.y *= w; vv.z *= w; vv.w *= w;
-                    const float *ki = kt + i * KDIM;
+                // newest token first, w_i = prod_{j>i} a_j; token i-1's key and value
+                // are read from shared memory while token i's products issue
+                float w = 1.f;
+                float4 vv = lds4(vt + (n - 1) * VS), kq[QROWS];
 #pragma unroll
-                    for (int q = 0; q < QROWS; ++q) quad_rank1(s + 4 * q, lds4(ki + q * 32), vv);
+                for (int q = 0; q < QROWS; ++q) kq[q] = lds4(kt + (n - 1) * KDIM + q * 32);
+                for (int i = n - 1; i >= 0; --i) {
+                    float4 vn = vv, kn[QROWS];
+#pragma unroll
+                    for (int q = 0; q < QROWS; ++q) kn[q] = kq[q];
+                    if (i > 0) {
+                        vn = lds4(vt + (i - 1) * VS);
+#pragma unroll
+                        for (int q = 0; q < QROWS; ++q) kn[q] = lds4(kt + (i - 1) * KDIM + q * 32);
+                    }
+                    vv.x *= w; vv.y *= w; vv.z *= w; vv.w *= w;
+#pragma unroll
+                    for (int q = 0; q < QROWS; ++q) quad_rank1(s + 4 * q, kq[q], vv);
                     w *= __shfl_sync(0xffffffffu, a_l, i);
+                    vv = vn;
+#pragma unroll
+                    for (int q = 0; q < QROWS; ++q) kq[q] = kn[q];
                 }
             }
         } else {
@@ -429,7 +447,7 @@ flush_kernel(const FlushArgs A)
                 }
                 o_phase ^= 1u;
             }
-            float *Yh = A.Y + ((long long)cur.b * A.rtot + __ldg(A.off + cur.h)) * V + (long long)cur.slab * VS +
+            float *Yh = A.Y + ((long long)cur.b * A.rtot + cur.off) * V + (long long)cur.slab * VS +
                         c4 * 4;
             const float *om = Obuf + 4 * ks;
             const bool u2 = ks & 4, u1 = ks & 2, u0 = ks & 1;
