@@ -455,6 +455,31 @@ def run_reference(args, cfg) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args, cfg) -> None:
+    """A small single-layer run for a profiler (ncu -k <kernel> -s <skip> -c <count>):
+    flush(0), then `--steps` window cycles of W sketch decodes and a flush, with no timing
+    and no JSON line.  Launch order: the initial flush, then per cycle W x (products
+    kernel, combine kernel) and the flush."""
+    import torch
+    import rank_state_read_b200 as rs
+    rank = synth.layer_rank_table(cfg)
+    layer = rs.SketchLayer(cfg.kind, batch=cfg.B, heads=cfg.H, qk_heads=cfg.Hqk, key_dim=cfg.K,
+                           value_dim=cfg.V, window=cfg.W, groups=cfg.G, rank_cap=cfg.cap,
+                           rank=rank.tolist(), omega=synth.basis(cfg),
+                           S0=synth.device_state(cfg, replica_seed(0, 0), "cuda"), device="cuda")
+    xs = [synth.device_step_inputs(cfg, 1000 + p, "cuda") for p in range(cfg.W)]
+    layer.flush(0)
+    for _ in range(args.steps):
+        for p in range(cfg.W):
+            x = xs[p]
+            layer.decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
+        layer.flush(cfg.W)
+    torch.cuda.synchronize()
+    layer.plan.check()
+    layer.close()
+    print(f"profile case done: config {args.config}, {args.steps} window cycle(s)", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -465,7 +490,12 @@ def main():
     ap.add_argument("--replicas", type=int, default=8)
     ap.add_argument("--ref-rows", type=int, default=32)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--profile", action="store_true",
+                    help="small single-layer run for a profiler: no timing, no JSON line")
     args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args, synth.config(args.config))
+        return
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     cfg = synth.config(args.config)
