@@ -14,18 +14,27 @@
 // Work item: (b, h, column slab of VS columns); columns of S evolve independently,
 // so a slab is self-contained.  A persistent CTA walks a contiguous range of items
 // (consecutive heads of a batch row) with VS/16 compute warps and one producer warp.
-// Compute thread (ks, c4) holds the float4 column chunk c4 of the 16 state rows
-// 4 ks + 32 q + e (q, e < 4); a warp covers 4 column chunks x 8 row slices, so every
-// reduction over k (the delta-rule erase term k^T S and the projection Omega S) stays
-// inside the warp, and the float4 reads of keys, decays and basis rows by the 8 row
-// slices are 128 consecutive bytes (no bank conflict, no padding).
+// Each compute warp owns 16 columns of the slab and holds them for all 128 state rows
+// in registers (64 fp32 a thread).
+//   Mamba-2: the rank-n update S <- P S + K^T (w o V) runs on the tensor cores
+//   (mma.sync m16n8k8, tf32 operands split as x = hi + lo with the three products
+//   hi hi + hi lo + lo hi, which keeps fp32 accuracy); the state lives in the
+//   accumulator layout (columns 8 nt + 2 t (+1) for lane 4 g + t, and a fixed map of
+//   accumulator rows to state rows that keeps the fragment reads of the padded 4-row
+//   chunks conflict-free).  Key and value rows are staged with 8 floats of padding.
+//   GDN / KDA: thread (ks, c4) holds the float4 column chunk c4 of the 16 state rows
+//   4 ks + 32 q + e (q, e < 4) and applies the delta rule token by token; every
+//   reduction over k stays inside the warp, and the float4 reads of keys and decays by
+//   the 8 row slices are 128 consecutive bytes.
+// Both then project the new state onto the basis rows on the FP32 pipe and write S and
+// the sketch rows straight from registers.
 //
 // Data movement is TMA bulk copies (cp.async.bulk, completion counted on an mbarrier),
 // which keep far more bytes in flight per SM than register loads.  The producer warp
 // requests, one item ahead:
 //   - the item's state slab into one shared buffer, as 32 chunks of 4 rows, each
-//     chunk padded by 4 floats so that the 8 row slices' float4 reads fall on
-//     disjoint banks;
+//     chunk padded by 4 floats (so that the reads of all threads of a warp fall on
+//     disjoint banks);
 //   - the buffered keys, values and KDA decays into one of two token buffers;
 //   - when the head group changes, the basis rows 0 .. rmax_g - 1 of the new group,
 //     which stay resident while the group lasts.
@@ -48,16 +57,25 @@ constexpr int FLUSH_MAXT = 192;   // up to 5 compute warps (VS <= 80) + the prod
 struct FlushCarve {
     size_t bar, S, T, O, total;          // byte offsets in shared memory
     size_t tkeys, tv, ta, tfloats;       // float offsets within one token buffer
+    int ks, vs;                          // row strides (floats) of staged keys and values
 };
+
+// Mamba-2 token rows are staged padded: values by 8 floats (the B-fragment reads of 4
+// tokens x 8 columns hit 32 distinct banks), keys by 4 (the A-fragment reads of 4 tokens
+// x 8 state rows spaced 8 apart hit 8 banks, 4 lanes each)
+constexpr int MPAD_V = 8, MPAD_K = 4;
 
 __host__ __device__ inline size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
 
 __host__ __device__ inline FlushCarve flush_carve(int kind, int VS, int W, int rcap)
 {
     FlushCarve c;
+    const bool m2 = kind == SKETCHSSM_MAMBA2;
+    c.ks = m2 ? KDIM + MPAD_K : KDIM;
+    c.vs = m2 ? VS + MPAD_V : VS;
     c.tkeys = 0;
-    c.tv = (size_t)W * KDIM;
-    c.ta = c.tv + (size_t)W * VS;
+    c.tv = (size_t)W * c.ks;
+    c.ta = c.tv + (size_t)W * c.vs;
     c.tfloats = c.ta + (kind == SKETCHSSM_KDA ? (size_t)W * KDIM : 0);
     size_t o = 0;
     c.bar = o;  // full, empty, omega barriers and the abort flag
@@ -144,6 +162,16 @@ __device__ __forceinline__ void issue_item(const FlushArgs &A, const Cursor &it,
         for (int e = 0; e < 4; ++e)
             bulk_copy_g2s(dst + e * VS, Sg + (long long)(lane * 4 + e) * V, (uint32_t)(4 * VS), bar);
     }
+    if (KIND == SKETCHSSM_MAMBA2) {  // keys and values one padded row each
+        if (n > 0 && lane < n) {
+            const int qk = it.h / A.hpq;
+            bulk_copy_g2s(T + cv.tkeys + (size_t)lane * cv.ks,
+                          A.kbuf + (((long long)it.b * A.Hqk + qk) * W + lane) * KDIM, (uint32_t)(KDIM * 4), bar);
+            bulk_copy_g2s(T + cv.tv + (size_t)lane * cv.vs, A.vbuf + (bh * W + lane) * V + (long long)it.slab * VS,
+                          (uint32_t)(VS * 4), bar);
+        }
+        return;
+    }
     if (n > 0) {
         const int qk = it.h / A.hpq;
         if (lane == 0)
@@ -189,6 +217,42 @@ __device__ __forceinline__ float4 shfl_xor4(float4 v, int m)
     return make_float4(__shfl_xor_sync(0xffffffffu, v.x, m), __shfl_xor_sync(0xffffffffu, v.y, m),
                        __shfl_xor_sync(0xffffffffu, v.z, m), __shfl_xor_sync(0xffffffffu, v.w, m));
 }
+
+// x = hi + lo with hi, lo tf32 (round to nearest, ties away): hi carries the top 11
+// significant bits, lo the next 11, so hi hi + hi lo + lo hi misses only lo lo
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
+{
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+    const float rest = x - __uint_as_float(hi);
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(rest));
+}
+
+// d += a b for one 16 x 8 x 8 tf32 tile (fp32 accumulate), fragments as in the PTX ISA
+// (lane 4 g + t: a = A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]; b = B[t][g], B[t+4][g];
+// d = D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1])
+__device__ __forceinline__ void mma_tf32(float *d, const uint32_t *a, const uint32_t *b)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Mamba-2 tensor-core row map: accumulator row 16 mt + g + 8 h holds state row
+//   srow = 8 g + 4 h + 64 (mt / 4) + mt % 4,
+// i.e. 4-row chunk 2 g + h + 16 (mt / 4), row mt % 4 of it.  In the padded chunk layout
+// of the slab buffer (chunk c at c (4 VS + 4), row e at e VS) the 4 rows g = 0..3 that a
+// half-warp reads together then start 8 banks apart: the float2 fragment reads are free
+// of bank conflicts.  Keys and basis rows are indexed with the same map.
+__device__ __forceinline__ int srow(int mt, int g, int h) { return 8 * g + 4 * h + 64 * (mt >> 2) + (mt & 3); }
+__device__ __forceinline__ int slab_off(int mt, int g, int h, int VS)
+{
+    return (2 * g + h + 16 * (mt >> 2)) * (4 * VS + 4) + (mt & 3) * VS;
+}
+
+__device__ __forceinline__ float2 lds2(const float *p) { return *reinterpret_cast<const float2 *>(p); }
+__device__ __forceinline__ void st2(float *p, float a, float b) { *reinterpret_cast<float2 *>(p) = make_float2(a, b); }
 
 // One step of a reduce-scatter between lanes that differ in bit `m`: the lane with
 // the bit clear keeps lo (adds the partner's lo), the other keeps hi.
@@ -305,6 +369,170 @@ flush_kernel(const FlushArgs A)
     load_scalars(cur, a_l, b_l);
     uint32_t o_phase = 0;
 
+    if constexpr (KIND == SKETCHSSM_MAMBA2) {
+        // ------------------------------------------------ Mamba-2 on the tensor cores
+        const int g = lane >> 2, t = lane & 3;
+        const int col0 = warp * 16;  // the warp's 16 columns of the slab
+        for (int j = 0; j < cnt; ++j) {
+            const float *T = Tb + (size_t)(j & 1) * cv.tfloats;
+            const int r = cur.r;
+            const bool need_o = new_group(cur);
+            if (!wait_or_abort(full, (uint32_t)(j & 1), A.wait_limit, abort)) {
+                if (lane == 0) {
+                    *abort = 1;
+                    atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
+                }
+                return;
+            }
+            // the state in the accumulator layout: c[mt][nt][2 h + e] = state row
+            // srow(mt, g, h), column col0 + 8 nt + 2 t + e
+            float c[8][2][4];
+            {
+                const float *sb = Sbuf + col0 + 2 * t;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const float2 lo = lds2(sb + slab_off(mt, g, 0, VS) + 8 * nt);
+                        const float2 hi = lds2(sb + slab_off(mt, g, 1, VS) + 8 * nt);
+                        c[mt][nt][0] = lo.x;
+                        c[mt][nt][1] = lo.y;
+                        c[mt][nt][2] = hi.x;
+                        c[mt][nt][3] = hi.y;
+                    }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty);
+
+            Cursor nxt = cur;
+            float a_n = 1.f, b_n = 0.f;
+            if (j + 1 < cnt) {
+                nxt.next(A, nslab);
+                load_scalars(nxt, a_n, b_n);
+            }
+
+            if (n > 0) {
+                // suffix products over the tokens (lanes >= n hold a = 1):
+                // x_i = prod_{j >= i} a_j, P = x_0, w_i = x_{i+1} = prod_{j > i} a_j
+                float x = a_l;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_down_sync(0xffffffffu, x, o);
+                    if (lane + o < 32) x *= y;
+                }
+                const float P = __shfl_sync(0xffffffffu, x, 0);
+                float wl = __shfl_down_sync(0xffffffffu, x, 1);
+                if (lane == 31) wl = 1.f;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) c[mt][nt][e] *= P;
+                // S += K^T (w o V), 8 tokens per k-step; tokens >= n contribute 0
+                const float *kt = T + cv.tkeys;
+                const float *vt = T + cv.tv + col0 + g;
+                for (int k0 = 0; k0 < n; k0 += 8) {
+                    const int i0 = k0 + t, i1 = k0 + t + 4;
+                    const bool ok0 = i0 < n, ok1 = i1 < n;
+                    const float w0 = __shfl_sync(0xffffffffu, wl, i0 & 31);
+                    const float w1 = __shfl_sync(0xffffffffu, wl, i1 & 31);
+                    uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const float v0 = ok0 ? w0 * vt[(size_t)i0 * cv.vs + 8 * nt] : 0.f;
+                        const float v1 = ok1 ? w1 * vt[(size_t)i1 * cv.vs + 8 * nt] : 0.f;
+                        split_tf32(v0, bh[nt][0], bl[nt][0]);
+                        split_tf32(v1, bh[nt][1], bl[nt][1]);
+                    }
+                    const float *k0p = kt + (size_t)i0 * cv.ks;
+                    const float *k1p = kt + (size_t)i1 * cv.ks;
+#pragma unroll
+                    for (int mt = 0; mt < 8; ++mt) {
+                        const int r0 = srow(mt, g, 0), r1 = srow(mt, g, 1);
+                        const float a0 = ok0 ? k0p[r0] : 0.f;
+                        const float a1 = ok0 ? k0p[r1] : 0.f;
+                        const float a2 = ok1 ? k1p[r0] : 0.f;
+                        const float a3 = ok1 ? k1p[r1] : 0.f;
+                        uint32_t ah[4], al[4];
+                        split_tf32(a0, ah[0], al[0]);
+                        split_tf32(a1, ah[1], al[1]);
+                        split_tf32(a2, ah[2], al[2]);
+                        split_tf32(a3, ah[3], al[3]);
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt) {
+                            mma_tf32(c[mt][nt], al, bh[nt]);
+                            mma_tf32(c[mt][nt], ah, bl[nt]);
+                            mma_tf32(c[mt][nt], ah, bh[nt]);
+                        }
+                    }
+                }
+                float *Sg = A.S + cur.bh(A) * KDIM * V + (long long)cur.slab * VS + col0 + 2 * t;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        st2(Sg + (long long)srow(mt, g, 0) * V + 8 * nt, c[mt][nt][0], c[mt][nt][1]);
+                        st2(Sg + (long long)srow(mt, g, 1) * V + 8 * nt, c[mt][nt][2], c[mt][nt][3]);
+                    }
+            }
+
+            // the sketch rows of the warp's columns, 8 at a time: partial sums over the
+            // thread's 16 state rows, then a reduce-scatter over g (lane bits 2..4)
+            // leaves sketch row m0 + g in lane 4 g + t
+            if (r > 0) {
+                if (need_o) {
+                    if (!wait_or_abort(obar, o_phase, A.wait_limit, abort)) {
+                        if (lane == 0) {
+                            *abort = 1;
+                            atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
+                        }
+                        return;
+                    }
+                    o_phase ^= 1u;
+                }
+                float *Yh = A.Y + ((long long)cur.b * A.rtot + cur.off) * V + (long long)cur.slab * VS + col0 + 2 * t;
+                const float *om = Obuf;
+                for (int m0 = 0; m0 < r; m0 += 8) {
+                    float4 p[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        float4 x0 = zero4(), x1 = zero4();
+                        if (m0 + u < r) {
+                            const float *o = om + (m0 + u) * KDIM;
+#pragma unroll
+                            for (int mt = 0; mt < 8; ++mt) {
+                                const float o0 = o[srow(mt, g, 0)], o1 = o[srow(mt, g, 1)];
+                                float4 &xx = (mt & 1) ? x1 : x0;
+                                xx.x = fmaf(o0, c[mt][0][0], xx.x);
+                                xx.y = fmaf(o0, c[mt][0][1], xx.y);
+                                xx.z = fmaf(o0, c[mt][1][0], xx.z);
+                                xx.w = fmaf(o0, c[mt][1][1], xx.w);
+                                xx.x = fmaf(o1, c[mt][0][2], xx.x);
+                                xx.y = fmaf(o1, c[mt][0][3], xx.y);
+                                xx.z = fmaf(o1, c[mt][1][2], xx.z);
+                                xx.w = fmaf(o1, c[mt][1][3], xx.w);
+                            }
+                        }
+                        p[u] = add4(x0, x1);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) p[u] = rs_step(p[u], p[u + 4], (lane & 16) != 0, 16);
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) p[u] = rs_step(p[u], p[u + 2], (lane & 8) != 0, 8);
+                    p[0] = rs_step(p[0], p[1], (lane & 4) != 0, 4);
+                    if (m0 + g < r) {
+                        float *y = Yh + (long long)(m0 + g) * V;
+                        st2(y, p[0].x, p[0].y);
+                        st2(y + 8, p[0].z, p[0].w);
+                    }
+                }
+            }
+            cur = nxt;
+            a_l = a_n;
+            b_l = b_n;
+        }
+    } else {
     for (int j = 0; j < cnt; ++j) {
         const float *T = Tb + (size_t)(j & 1) * cv.tfloats;
         const int r = cur.r;
@@ -476,6 +704,7 @@ flush_kernel(const FlushArgs A)
         cur = nxt;
         a_l = a_n;
         b_l = b_n;
+    }
     }
 }
 
