@@ -53,11 +53,11 @@ __host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
 // ============================================================================ query-side products
 
 constexpr int CM_THREADS = 256;
-constexpr int CM_MAXROWS = 8;
+constexpr int CM_MAXROWS = 4;
 constexpr int OPAD = KDIM + 4;  // padded row: threads reading different rows hit different banks
 
 struct CmCarve {
-    size_t om, ks, qs, sd, ud, total;
+    size_t om, qs, total;
 };
 
 __host__ __device__ inline size_t cm_take(size_t &o, size_t bytes)
@@ -69,117 +69,99 @@ __host__ __device__ inline size_t cm_take(size_t &o, size_t bytes)
 
 __host__ __device__ inline CmCarve cm_carve(int cap, int W, int rows)
 {
+    (void)W;
     CmCarve c;
     size_t o = 0;
     c.om = cm_take(o, sizeof(float) * (size_t)cap * OPAD);
-    c.ks = cm_take(o, sizeof(float) * (size_t)rows * W * OPAD);
-    c.qs = cm_take(o, sizeof(float) * (size_t)rows * KDIM);
-    c.sd = cm_take(o, sizeof(float) * (size_t)rows * W);
-    c.ud = cm_take(o, sizeof(float) * (size_t)rows * cap);
+    c.qs = cm_take(o, sizeof(float) * (size_t)rows * OPAD);
     c.total = o;
     return c;
 }
 
 // Mamba-2: one CTA per (q/k head, `rows` batch rows).  Output per (batch row, q/k
 // head): dots_row floats, s_0 .. s_{W-1} then u_0 .. u_{cap-1} (unused entries 0).
+//   s_i = k_i . q: one warp per (row, key), lanes over k, keys read straight from the
+//       buffer (each is used once), issued while the basis rows are being staged;
+//   u_m = Omega_g[m] . q: one thread per (basis row, batch row) over the staged rows
+//       (rows padded so that the 8 batch rows a quarter-warp reads hit 8 bank groups).
+// The step's key is appended to buffer slot pos.  The CTA needs a few KB of shared
+// memory, so the combine CTAs launched as its programmatic dependents fit beside it.
 __global__ void __launch_bounds__(CM_THREADS)
 dots_kernel_mamba2(const DecodeArgs A)
 {
     extern __shared__ __align__(128) unsigned char cms[];
     pdl_launch_dependents();  // the combine may start staging its rows now
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int W = A.W, pos = A.pos, n = pos + 1, hpq = A.hpq, cap = A.cap;
+    const int W = A.W, pos = A.pos, n = pos + 1, hpq = A.hpq, cap = A.cap, dr = A.dots_row;
     const int rows = A.cm_rows;
     const int q = blockIdx.x, b0 = blockIdx.y * rows;
     const int nb = min(rows, A.B - b0);
     const int g = (q * hpq) / A.Hg;
     const CmCarve cv = cm_carve(cap, W, rows);
-    float *om = reinterpret_cast<float *>(cms + cv.om);     // [cap][OPAD]
-    float *ks = reinterpret_cast<float *>(cms + cv.ks);     // [rows][W][OPAD] keys (slot pos: the step's)
-    float *qs = reinterpret_cast<float *>(cms + cv.qs);     // [rows][K]
-    float *s_dot = reinterpret_cast<float *>(cms + cv.sd);  // [rows][W]
-    float *u_dot = reinterpret_cast<float *>(cms + cv.ud);  // [rows][cap]
+    float *om = reinterpret_cast<float *>(cms + cv.om);  // [rq][OPAD]
+    float *qs = reinterpret_cast<float *>(cms + cv.qs);  // [rows][OPAD]
 
-    const int orows = A.dense_all ? 0 : cap;
+    const int rq = A.dense_all ? 0 : __ldg(A.qk_rneed + q);
     const float *og = A.omega + (long long)g * A.Rb * KDIM;
-    for (int x = tid; x < orows * (KDIM / 4); x += CM_THREADS) {
+    for (int x = tid; x < rq * (KDIM / 4); x += CM_THREADS) {
         const int j = x >> 5, c = x & 31;
         cp_async16(om + j * OPAD + c * 4, og + (long long)j * KDIM + c * 4);
     }
     for (int x = tid; x < nb * (KDIM / 4); x += CM_THREADS) {
         const int bl = x >> 5, c = x & 31;
-        cp_async16(qs + bl * KDIM + c * 4, A.q + ((long long)(b0 + bl) * A.Hqk + q) * KDIM + c * 4);
+        cp_async16(qs + bl * OPAD + c * 4, A.q + ((long long)(b0 + bl) * A.Hqk + q) * KDIM + c * 4);
     }
-    for (int x = tid; x < nb * n * (KDIM / 4); x += CM_THREADS) {
-        const int c = x & 31, r = x >> 5, bl = r / n, i = r - bl * n;
-        const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
-        cp_async16(ks + (bl * W + i) * OPAD + c * 4,
-                   (i == pos ? A.k + qrow * KDIM : A.kbuf + (qrow * W + i) * KDIM) + c * 4);
-    }
-    const int rq = A.dense_all ? 0 : __ldg(A.qk_rneed + q);
     cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
 
-    if (warp < 4) {
-        // u[bl][j] = Omega_g[j] . q_bl: thread j, all batch rows at once
-        for (int j = tid; j < rq; j += 128) {
-            const float *orow = om + (size_t)j * OPAD;
-            float acc[CM_MAXROWS];
+    // s: warp per (row, key), four in flight
+    constexpr int NWARP = CM_THREADS / 32;
+    for (int t0 = warp; t0 < nb * n; t0 += 4 * NWARP) {
+        float4 kv[4], qv[4];
 #pragma unroll
-            for (int bl = 0; bl < CM_MAXROWS; ++bl) acc[bl] = 0.f;
-#pragma unroll 4
-            for (int c = 0; c < KDIM; c += 4) {
-                const float4 o = lds4(orow + c);
-#pragma unroll
-                for (int bl = 0; bl < CM_MAXROWS; ++bl) {
-                    if (bl < nb) {
-                        const float4 x = lds4(qs + bl * KDIM + c);
-                        acc[bl] = fmaf(o.x, x.x, fmaf(o.y, x.y, fmaf(o.z, x.z, fmaf(o.w, x.w, acc[bl]))));
-                    }
-                }
+        for (int k = 0; k < 4; ++k) {
+            const int t = t0 + k * NWARP;
+            kv[k] = qv[k] = zero4();
+            if (t < nb * n) {
+                const int bl = t / n, i = t - bl * n;
+                const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
+                kv[k] = ldg4((i == pos ? A.k + qrow * KDIM : A.kbuf + (qrow * W + i) * KDIM) + lane * 4);
+                qv[k] = ldg4(A.q + qrow * KDIM + lane * 4);
             }
-#pragma unroll
-            for (int bl = 0; bl < CM_MAXROWS; ++bl)
-                if (bl < nb) u_dot[bl * cap + j] = acc[bl];
         }
-    } else {
-        // s[bl][i] = k_i . q_bl: a half warp per batch row, lane i per key
-        const int half = (warp - 4) * 2 + (lane >> 4), i0 = lane & 15;
-        for (int bl = half; bl < nb; bl += 8) {
-            const float *qb = qs + bl * KDIM;
-            for (int i = i0; i < n; i += 16) {
-                const float *row = ks + (bl * W + i) * OPAD;
-                float4 acc = zero4();
-#pragma unroll 8
-                for (int c = 0; c < KDIM; c += 4) {
-                    const float4 o = lds4(row + c), x = lds4(qb + c);
-                    acc.x = fmaf(o.x, x.x, acc.x);
-                    acc.y = fmaf(o.y, x.y, acc.y);
-                    acc.z = fmaf(o.z, x.z, acc.z);
-                    acc.w = fmaf(o.w, x.w, acc.w);
-                }
-                s_dot[bl * W + i] = (acc.x + acc.y) + (acc.z + acc.w);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int t = t0 + k * NWARP;
+            const float d = warp_sum(dot4(kv[k], qv[k]));
+            if (t < nb * n) {
+                const int bl = t / n, i = t - bl * n;
+                const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
+                if (lane == 0) A.scratch[qrow * dr + i] = d;
+                if (i == pos) st4(A.kbuf + (qrow * W + pos) * KDIM + lane * 4, kv[k]);
             }
         }
     }
-    // the step's key goes to buffer slot pos (from the stage)
-    for (int x = tid; x < nb * (KDIM / 4); x += CM_THREADS) {
-        const int bl = x >> 5, c = x & 31;
-        const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
-        st4(A.kbuf + (qrow * W + pos) * KDIM + c * 4, lds4(ks + (bl * W + pos) * OPAD + c * 4));
-    }
-    __syncthreads();
-    const int dr = A.dots_row;
+    // unused entries of the rows: 0
     for (int x = tid; x < nb * dr; x += CM_THREADS) {
         const int bl = x / dr, e = x - bl * dr;
-        float v = 0.f;
-        if (e < W) {
-            if (e < n) v = s_dot[bl * W + e];
-        } else if (e - W < rq) {
-            v = u_dot[bl * cap + (e - W)];
+        if ((e >= n && e < W) || e >= W + rq) A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + e] = 0.f;
+    }
+
+    cp_async_wait<0>();
+    __syncthreads();
+    // u: thread per (basis row, batch row), four partial sums
+    for (int x = tid; x < rq * nb; x += CM_THREADS) {
+        const int j = x / nb, bl = x - j * nb;
+        const float *orow = om + (size_t)j * OPAD, *qb = qs + (size_t)bl * OPAD;
+        float4 acc = zero4();
+#pragma unroll 8
+        for (int c = 0; c < KDIM; c += 4) {
+            const float4 o = lds4(orow + c), v = lds4(qb + c);
+            acc.x = fmaf(o.x, v.x, acc.x);
+            acc.y = fmaf(o.y, v.y, acc.y);
+            acc.z = fmaf(o.z, v.z, acc.z);
+            acc.w = fmaf(o.w, v.w, acc.w);
         }
-        A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + e] = v;
+        A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + W + j] = (acc.x + acc.y) + (acc.z + acc.w);
     }
 }
 
@@ -526,10 +508,9 @@ int coef_block(int rows, int W) { return round4(rows + W); }
 
 int coef_rows(int cap, int W)
 {
-    // batch rows per Mamba-2 product CTA: as many as keep two CTAs on an SM
-    for (int rows = CM_MAXROWS; rows > 1; rows >>= 1)
-        if (cm_carve(cap, W, rows).total <= 110 * 1024) return rows;
-    return 1;
+    (void)cap;
+    (void)W;
+    return CM_MAXROWS;  // batch rows per Mamba-2 product CTA
 }
 
 size_t decode_smem_bytes(const DecodeArgs &a)
