@@ -57,7 +57,9 @@ constexpr int CM_MAXROWS = 4;
 constexpr int OPAD = KDIM + 4;  // padded row: threads reading different rows hit different banks
 
 struct CmCarve {
-    size_t om, qs, total;
+    size_t om, qs, ks, total;
+    int kblock;  // floats per batch row of staged keys (W padded rows + 4: rows of different
+                 // batch rows start 4 banks apart)
 };
 
 __host__ __device__ inline size_t cm_take(size_t &o, size_t bytes)
@@ -69,29 +71,30 @@ __host__ __device__ inline size_t cm_take(size_t &o, size_t bytes)
 
 __host__ __device__ inline CmCarve cm_carve(int cap, int W, int rows)
 {
-    (void)W;
     CmCarve c;
+    c.kblock = W * OPAD + 4;
     size_t o = 0;
     c.om = cm_take(o, sizeof(float) * (size_t)cap * OPAD);
     c.qs = cm_take(o, sizeof(float) * (size_t)rows * OPAD);
+    c.ks = cm_take(o, sizeof(float) * (size_t)rows * c.kblock);
     c.total = o;
     return c;
 }
 
 // Mamba-2: one CTA per (q/k head, `rows` batch rows).  Output per (batch row, q/k
 // head): dots_row floats, s_0 .. s_{W-1} then u_0 .. u_{cap-1} (unused entries 0).
-//   s_i = k_i . q: one warp per (row, key), lanes over k, keys read straight from the
-//       buffer (each is used once), issued while the basis rows are being staged;
-//   u_m = Omega_g[m] . q: one thread per (basis row, batch row) over the staged rows
-//       (rows padded so that the 8 batch rows a quarter-warp reads hit 8 bank groups).
-// The step's key is appended to buffer slot pos.  The CTA needs a few KB of shared
-// memory, so the combine CTAs launched as its programmatic dependents fit beside it.
+// One round of cp.async stages the group's basis rows, the rows' queries and keys (the
+// step's key in slot pos); then every dot product s_i = k_i . q and u_m = Omega_g[m] . q
+// is one thread's loop over 128 staged floats.  Task t = (row t / rows, batch row
+// t % rows): the threads of a quarter-warp read one basis row (broadcast) or keys and
+// queries of different batch rows (padded to fall on different banks).  The step's key
+// is appended to buffer slot pos.
 __global__ void __launch_bounds__(CM_THREADS)
 dots_kernel_mamba2(const DecodeArgs A)
 {
     extern __shared__ __align__(128) unsigned char cms[];
     pdl_launch_dependents();  // the combine may start staging its rows now
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int W = A.W, pos = A.pos, n = pos + 1, hpq = A.hpq, cap = A.cap, dr = A.dots_row;
     const int rows = A.cm_rows;
     const int q = blockIdx.x, b0 = blockIdx.y * rows;
@@ -100,6 +103,7 @@ dots_kernel_mamba2(const DecodeArgs A)
     const CmCarve cv = cm_carve(cap, W, rows);
     float *om = reinterpret_cast<float *>(cms + cv.om);  // [rq][OPAD]
     float *qs = reinterpret_cast<float *>(cms + cv.qs);  // [rows][OPAD]
+    float *ks = reinterpret_cast<float *>(cms + cv.ks);  // [rows][kblock]: key i at i OPAD
 
     const int rq = A.dense_all ? 0 : __ldg(A.qk_rneed + q);
     const float *og = A.omega + (long long)g * A.Rb * KDIM;
@@ -111,57 +115,42 @@ dots_kernel_mamba2(const DecodeArgs A)
         const int bl = x >> 5, c = x & 31;
         cp_async16(qs + bl * OPAD + c * 4, A.q + ((long long)(b0 + bl) * A.Hqk + q) * KDIM + c * 4);
     }
-    cp_async_commit();
-
-    // s: warp per (row, key), four in flight
-    constexpr int NWARP = CM_THREADS / 32;
-    for (int t0 = warp; t0 < nb * n; t0 += 4 * NWARP) {
-        float4 kv[4], qv[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int t = t0 + k * NWARP;
-            kv[k] = qv[k] = zero4();
-            if (t < nb * n) {
-                const int bl = t / n, i = t - bl * n;
-                const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
-                kv[k] = ldg4((i == pos ? A.k + qrow * KDIM : A.kbuf + (qrow * W + i) * KDIM) + lane * 4);
-                qv[k] = ldg4(A.q + qrow * KDIM + lane * 4);
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int t = t0 + k * NWARP;
-            const float d = warp_sum(dot4(kv[k], qv[k]));
-            if (t < nb * n) {
-                const int bl = t / n, i = t - bl * n;
-                const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
-                if (lane == 0) A.scratch[qrow * dr + i] = d;
-                if (i == pos) st4(A.kbuf + (qrow * W + pos) * KDIM + lane * 4, kv[k]);
-            }
-        }
+    for (int x = tid; x < nb * n * (KDIM / 4); x += CM_THREADS) {
+        const int c = x & 31, r = x >> 5, bl = r / n, i = r - bl * n;
+        const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
+        cp_async16(ks + bl * cv.kblock + i * OPAD + c * 4,
+                   (i == pos ? A.k + qrow * KDIM : A.kbuf + (qrow * W + i) * KDIM) + c * 4);
     }
+    cp_async_commit();
     // unused entries of the rows: 0
     for (int x = tid; x < nb * dr; x += CM_THREADS) {
         const int bl = x / dr, e = x - bl * dr;
         if ((e >= n && e < W) || e >= W + rq) A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + e] = 0.f;
     }
-
     cp_async_wait<0>();
     __syncthreads();
-    // u: thread per (basis row, batch row), four partial sums
-    for (int x = tid; x < rq * nb; x += CM_THREADS) {
-        const int j = x / nb, bl = x - j * nb;
-        const float *orow = om + (size_t)j * OPAD, *qb = qs + (size_t)bl * OPAD;
+
+    for (int t = tid; t < (n + rq) * nb; t += CM_THREADS) {
+        const int rr = t / nb, bl = t - rr * nb;
+        const float *row = rr < n ? ks + bl * cv.kblock + rr * OPAD : om + (size_t)(rr - n) * OPAD;
+        const float *qb = qs + (size_t)bl * OPAD;
         float4 acc = zero4();
 #pragma unroll 8
         for (int c = 0; c < KDIM; c += 4) {
-            const float4 o = lds4(orow + c), v = lds4(qb + c);
+            const float4 o = lds4(row + c), v = lds4(qb + c);
             acc.x = fmaf(o.x, v.x, acc.x);
             acc.y = fmaf(o.y, v.y, acc.y);
             acc.z = fmaf(o.z, v.z, acc.z);
             acc.w = fmaf(o.w, v.w, acc.w);
         }
-        A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + W + j] = (acc.x + acc.y) + (acc.z + acc.w);
+        A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + (rr < n ? rr : W + rr - n)] =
+            (acc.x + acc.y) + (acc.z + acc.w);
+    }
+    // the step's key goes to buffer slot pos (from the stage)
+    for (int x = tid; x < nb * (KDIM / 4); x += CM_THREADS) {
+        const int bl = x >> 5, c = x & 31;
+        const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
+        st4(A.kbuf + (qrow * W + pos) * KDIM + c * 4, lds4(ks + bl * cv.kblock + pos * OPAD + c * 4));
     }
 }
 
