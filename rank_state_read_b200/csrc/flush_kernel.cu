@@ -55,7 +55,7 @@ constexpr int QROWS = KDIM / 32;  // row quads per thread (4): rows 4 ks + 32 q 
 constexpr int FLUSH_MAXT = 192;   // up to 5 compute warps (VS <= 80) + the producer
 
 struct FlushCarve {
-    size_t bar, S, T, O, total;          // byte offsets in shared memory
+    size_t bar, S, T, O, AF, total;      // byte offsets in shared memory
     size_t tkeys, tv, ta, tfloats;       // float offsets within one token buffer
     int ks, vs;                          // row strides (floats) of staged keys and values
 };
@@ -86,6 +86,8 @@ __host__ __device__ inline FlushCarve flush_carve(int kind, int VS, int W, int r
     o = align128(o + 2 * sizeof(float) * c.tfloats);
     c.O = o;
     o = align128(o + sizeof(float) * (size_t)rcap * KDIM);
+    c.AF = o;  // Mamba-2: split key fragments, [k-step][m-tile][lane][hi 4, lo 4]
+    o = align128(o + (m2 ? sizeof(float) * (size_t)((W + 7) / 8) * 8 * 32 * 8 : 0));
     c.total = o;
     return c;
 }
@@ -254,6 +256,12 @@ __device__ __forceinline__ int slab_off(int mt, int g, int h, int VS)
 __device__ __forceinline__ float2 lds2(const float *p) { return *reinterpret_cast<const float2 *>(p); }
 __device__ __forceinline__ void st2(float *p, float a, float b) { *reinterpret_cast<float2 *>(p) = make_float2(a, b); }
 
+// named barrier 1 among the compute warps (the producer warp does not take part)
+__device__ __forceinline__ void compute_barrier(int ncw)
+{
+    asm volatile("bar.sync 1, %0;" ::"r"(ncw * 32) : "memory");
+}
+
 // One step of a reduce-scatter between lanes that differ in bit `m`: the lane with
 // the bit clear keeps lo (adds the partner's lo), the other keeps hi.
 __device__ __forceinline__ float4 rs_step(float4 lo, float4 hi, bool upper, int m)
@@ -373,17 +381,14 @@ flush_kernel(const FlushArgs A)
         // ------------------------------------------------ Mamba-2 on the tensor cores
         const int g = lane >> 2, t = lane & 3;
         const int col0 = warp * 16;  // the warp's 16 columns of the slab
+        float *AF = reinterpret_cast<float *>(fsm_raw + cv.AF);
+        long long af_key = -1;  // (b, q/k head) whose keys the fragment cache holds
+        bool ok = true;         // false once a wait gave up: no more work, barriers only
         for (int j = 0; j < cnt; ++j) {
             const float *T = Tb + (size_t)(j & 1) * cv.tfloats;
             const int r = cur.r;
             const bool need_o = new_group(cur);
-            if (!wait_or_abort(full, (uint32_t)(j & 1), A.wait_limit, abort)) {
-                if (lane == 0) {
-                    *abort = 1;
-                    atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
-                }
-                return;
-            }
+            ok = ok && wait_or_abort(full, (uint32_t)(j & 1), A.wait_limit, abort);
             // the state in the accumulator layout: c[mt][nt][2 h + e] = state row
             // srow(mt, g, h), column col0 + 8 nt + 2 t + e
             float c[8][2][4];
@@ -429,8 +434,28 @@ flush_kernel(const FlushArgs A)
                     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                         for (int e = 0; e < 4; ++e) c[mt][nt][e] *= P;
+                // the keys' A fragments, split hi / lo once per key set (shared by the
+                // heads of a q/k head): all compute warps build them between two named
+                // barriers; tokens >= n are 0
+                const long long key = (long long)cur.b * A.Hqk + cur.h / A.hpq;
+                if (key != af_key) {
+                    af_key = key;
+                    compute_barrier(ncw);  // every warp is done with the previous set
+                    const int nkt = (n + 7) >> 3;
+                    const float *kt = T + cv.tkeys;
+                    for (int x = warp * 32 + lane; x < nkt * 8 * 32 * 4; x += ncw * 32) {
+                        const int comp = x & 3, ln = (x >> 2) & 31, mt = (x >> 7) & 7, k8 = x >> 10;
+                        const int tok = 8 * k8 + (ln & 3) + 4 * (comp >> 1);
+                        const float v = (ok && tok < n) ? kt[(size_t)tok * cv.ks + srow(mt, ln >> 2, comp & 1)] : 0.f;
+                        uint32_t hi, lo;
+                        split_tf32(v, hi, lo);
+                        float *f = AF + (size_t)((k8 * 8 + mt) * 32 + ln) * 8;
+                        f[comp] = __uint_as_float(hi);
+                        f[4 + comp] = __uint_as_float(lo);
+                    }
+                    compute_barrier(ncw);
+                }
                 // S += K^T (w o V), 8 tokens per k-step; tokens >= n contribute 0
-                const float *kt = T + cv.tkeys;
                 const float *vt = T + cv.tv + col0 + g;
                 for (int k0 = 0; k0 < n; k0 += 8) {
                     const int i0 = k0 + t, i1 = k0 + t + 4;
@@ -445,20 +470,12 @@ flush_kernel(const FlushArgs A)
                         split_tf32(v0, bh[nt][0], bl[nt][0]);
                         split_tf32(v1, bh[nt][1], bl[nt][1]);
                     }
-                    const float *k0p = kt + (size_t)i0 * cv.ks;
-                    const float *k1p = kt + (size_t)i1 * cv.ks;
+                    const float *af = AF + (size_t)((k0 >> 3) * 8 * 32 + lane) * 8;
 #pragma unroll
                     for (int mt = 0; mt < 8; ++mt) {
-                        const int r0 = srow(mt, g, 0), r1 = srow(mt, g, 1);
-                        const float a0 = ok0 ? k0p[r0] : 0.f;
-                        const float a1 = ok0 ? k0p[r1] : 0.f;
-                        const float a2 = ok1 ? k1p[r0] : 0.f;
-                        const float a3 = ok1 ? k1p[r1] : 0.f;
-                        uint32_t ah[4], al[4];
-                        split_tf32(a0, ah[0], al[0]);
-                        split_tf32(a1, ah[1], al[1]);
-                        split_tf32(a2, ah[2], al[2]);
-                        split_tf32(a3, ah[3], al[3]);
+                        const uint4 fh = *reinterpret_cast<const uint4 *>(af + mt * 32 * 8);
+                        const uint4 fl = *reinterpret_cast<const uint4 *>(af + mt * 32 * 8 + 4);
+                        const uint32_t ah[4] = {fh.x, fh.y, fh.z, fh.w}, al[4] = {fl.x, fl.y, fl.z, fl.w};
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt) {
                             mma_tf32(c[mt][nt], al, bh[nt]);
@@ -468,29 +485,25 @@ flush_kernel(const FlushArgs A)
                     }
                 }
                 float *Sg = A.S + cur.bh(A) * KDIM * V + (long long)cur.slab * VS + col0 + 2 * t;
+                if (ok) {
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt)
+                    for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        st2(Sg + (long long)srow(mt, g, 0) * V + 8 * nt, c[mt][nt][0], c[mt][nt][1]);
-                        st2(Sg + (long long)srow(mt, g, 1) * V + 8 * nt, c[mt][nt][2], c[mt][nt][3]);
-                    }
+                        for (int nt = 0; nt < 2; ++nt) {
+                            st2(Sg + (long long)srow(mt, g, 0) * V + 8 * nt, c[mt][nt][0], c[mt][nt][1]);
+                            st2(Sg + (long long)srow(mt, g, 1) * V + 8 * nt, c[mt][nt][2], c[mt][nt][3]);
+                        }
+                }
             }
 
             // the sketch rows of the warp's columns, 8 at a time: partial sums over the
             // thread's 16 state rows, then a reduce-scatter over g (lane bits 2..4)
             // leaves sketch row m0 + g in lane 4 g + t
-            if (r > 0) {
-                if (need_o) {
-                    if (!wait_or_abort(obar, o_phase, A.wait_limit, abort)) {
-                        if (lane == 0) {
-                            *abort = 1;
-                            atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
-                        }
-                        return;
-                    }
-                    o_phase ^= 1u;
-                }
+            if (need_o) {
+                ok = ok && wait_or_abort(obar, o_phase, A.wait_limit, abort);
+                o_phase ^= 1u;
+            }
+            if (r > 0 && ok) {
                 float *Yh = A.Y + ((long long)cur.b * A.rtot + cur.off) * V + (long long)cur.slab * VS + col0 + 2 * t;
                 const float *om = Obuf;
                 for (int m0 = 0; m0 < r; m0 += 8) {
@@ -531,6 +544,10 @@ flush_kernel(const FlushArgs A)
             cur = nxt;
             a_l = a_n;
             b_l = b_n;
+        }
+        if (!ok && lane == 0) {
+            *abort = 1;
+            atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
         }
     } else {
     for (int j = 0; j < cnt; ++j) {
