@@ -137,16 +137,17 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, lo
 // on the barrier with no bytes.
 template <int KIND>
 __device__ __forceinline__ void issue_item(const FlushArgs &A, const Cursor &it, int nslab, float *Sbuf,
-                                           float *T, const FlushCarve &cv, uint64_t *bar, int lane)
+                                           float *T, const FlushCarve &cv, uint64_t *bar, int lane, bool keys)
 {
     const int V = A.V, VS = A.VS, W = A.W, n = A.n;
     const bool needed = n > 0 || it.r > 0;
+    if (KIND != SKETCHSSM_MAMBA2) keys = true;
     if (lane == 0) {
         uint32_t bytes = 0;
         if (needed) {
             bytes = (uint32_t)(KDIM * VS * 4);
             if (n > 0) {
-                bytes += (uint32_t)(n * KDIM * 4 + n * VS * 4);
+                bytes += (uint32_t)((keys ? n * KDIM * 4 : 0) + n * VS * 4);
                 if (KIND == SKETCHSSM_KDA) bytes += (uint32_t)(n * KDIM * 4);
             }
         }
@@ -164,11 +165,12 @@ __device__ __forceinline__ void issue_item(const FlushArgs &A, const Cursor &it,
         for (int e = 0; e < 4; ++e)
             bulk_copy_g2s(dst + e * VS, Sg + (long long)(lane * 4 + e) * V, (uint32_t)(4 * VS), bar);
     }
-    if (KIND == SKETCHSSM_MAMBA2) {  // keys and values one padded row each
+    if (KIND == SKETCHSSM_MAMBA2) {  // keys (only for a new key set) and values, one padded row each
         if (n > 0 && lane < n) {
             const int qk = it.h / A.hpq;
-            bulk_copy_g2s(T + cv.tkeys + (size_t)lane * cv.ks,
-                          A.kbuf + (((long long)it.b * A.Hqk + qk) * W + lane) * KDIM, (uint32_t)(KDIM * 4), bar);
+            if (keys)
+                bulk_copy_g2s(T + cv.tkeys + (size_t)lane * cv.ks,
+                              A.kbuf + (((long long)it.b * A.Hqk + qk) * W + lane) * KDIM, (uint32_t)(KDIM * 4), bar);
             bulk_copy_g2s(T + cv.tv + (size_t)lane * cv.vs, A.vbuf + (bh * W + lane) * V + (long long)it.slab * VS,
                           (uint32_t)(VS * 4), bar);
         }
@@ -329,9 +331,12 @@ flush_kernel(const FlushArgs A)
             last_o = (uint32_t)(issued_o & 1);
             ++issued_o;
         };
+        // Mamba-2 copies an item's keys only when its key set (b, q/k head) changes: the
+        // compute warps read them once, into the fragment cache
+        long long pk = (long long)cur.b * A.Hqk + cur.h / A.hpq;
         bool pend_o = new_group(cur);
         if (pend_o) o_rows = __ldg(A.rmax + cur.h / A.Hg);
-        issue_item<KIND>(A, cur, nslab, Sbuf, Tb, cv, full, lane);
+        issue_item<KIND>(A, cur, nslab, Sbuf, Tb, cv, full, lane, true);
         if (pend_o) issue_omega(cur);
         pend_o = false;
         bool ok = true;
@@ -345,7 +350,9 @@ flush_kernel(const FlushArgs A)
             cur.next(A, nslab);
             pend_o = new_group(cur);
             if (pend_o) o_rows = __ldg(A.rmax + cur.h / A.Hg);  // used one iteration later
-            issue_item<KIND>(A, cur, nslab, Sbuf, Tb + (size_t)(j & 1) * cv.tfloats, cv, full, lane);
+            const long long key = (long long)cur.b * A.Hqk + cur.h / A.hpq;
+            issue_item<KIND>(A, cur, nslab, Sbuf, Tb + (size_t)(j & 1) * cv.tfloats, cv, full, lane, key != pk);
+            pk = key;
             last_full = (uint32_t)(j & 1);
         }
         if (!ok) {
@@ -512,10 +519,17 @@ flush_kernel(const FlushArgs A)
                     for (int u = 0; u < 8; ++u) {
                         float4 x0 = zero4(), x1 = zero4();
                         if (m0 + u < r) {
-                            const float *o = om + (m0 + u) * KDIM;
+                            // the thread's 16 rows 8 g + 4 h + 64 (mt / 4) + mt % 4 are two
+                            // runs of 8 floats: four float4 reads
+                            const float *o = om + (m0 + u) * KDIM + 8 * g;
+                            const float4 oq[4] = {lds4(o), lds4(o + 4), lds4(o + 64), lds4(o + 68)};
+                            const float ov[4][4] = {{oq[0].x, oq[0].y, oq[0].z, oq[0].w},
+                                                    {oq[1].x, oq[1].y, oq[1].z, oq[1].w},
+                                                    {oq[2].x, oq[2].y, oq[2].z, oq[2].w},
+                                                    {oq[3].x, oq[3].y, oq[3].z, oq[3].w}};
 #pragma unroll
                             for (int mt = 0; mt < 8; ++mt) {
-                                const float o0 = o[srow(mt, g, 0)], o1 = o[srow(mt, g, 1)];
+                                const float o0 = ov[2 * (mt >> 2)][mt & 3], o1 = ov[2 * (mt >> 2) + 1][mt & 3];
                                 float4 &xx = (mt & 1) ? x1 : x0;
                                 xx.x = fmaf(o0, c[mt][0][0], xx.x);
                                 xx.y = fmaf(o0, c[mt][0][1], xx.y);
