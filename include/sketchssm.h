@@ -40,8 +40,8 @@
  *    launch; a call that returns an error launched nothing and wrote nothing.  A
  *    failed launch returns SKETCHSSM_ERR_CUDA; sketchssm_last_error() then gives
  *    the CUDA error text.  No call allocates or frees caller memory.  No kernel
- *    waits on another CTA; a decode CTA waits, with a bound, only for its own bulk
- *    copies, and records a timeout that sketchssm_plan_check reports.
+ *    waits on another CTA; a decode or flush CTA waits, with a bound, only for its
+ *    own bulk copies, and records a timeout that sketchssm_plan_check reports.
  *  - Decode / flush protocol: pos counts the tokens buffered since the last flush.
  *    sketchssm_decode(pos) appends the step's token at buffer slot pos and returns
  *    y including it.  After the decode at pos = W-1 the caller runs
@@ -68,7 +68,7 @@ typedef enum {
     SKETCHSSM_ERR_ALIGNMENT = 2,    /* a tensor pointer is not 16-byte aligned */
     SKETCHSSM_ERR_UNSUPPORTED = 3,  /* valid, but outside the shapes built for */
     SKETCHSSM_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
-    SKETCHSSM_ERR_TIMEOUT = 5       /* a kernel gave up a bounded wait (sketchssm_plan_check) */
+    SKETCHSSM_ERR_TIMEOUT = 5       /* a kernel wait ran past its limit (sketchssm_plan_check) */
 } sketchssm_status;
 
 typedef enum {
@@ -130,12 +130,24 @@ sketchssm_status sketchssm_plan_query(const sketchssm_plan *plan, int64_t *r_tot
 
 /*
  * Synchronise `stream`, then report what the kernels recorded on the plan since the
- * last check, and clear it: SKETCHSSM_ERR_TIMEOUT if a decode CTA gave up waiting
- * (about a second) for its own bulk copies, in which case that call's y is
- * incomplete; SKETCHSSM_OK otherwise.  No kernel waits on anything but its own
- * copies, so a timeout means a fault of the copy engine, not a deadlock.
+ * last check, and clear it: SKETCHSSM_ERR_TIMEOUT if a decode or flush CTA waited
+ * longer than the plan's wait limit (sketchssm_plan_set_wait_limit; default about a
+ * second) for its own bulk copies; SKETCHSSM_OK otherwise.  Such a CTA records the
+ * timeout and keeps waiting, up to the default limit more, for the same copies, so
+ * the outputs are complete unless that second wait also ran out (then the CTA gives
+ * up and its outputs are incomplete).  No kernel waits on anything but its own copies,
+ * so a timeout at the default limit means a fault of the copy engine, not a deadlock.
  */
 sketchssm_status sketchssm_plan_check(const sketchssm_plan *plan, sketchssm_stream stream);
+
+/*
+ * Set the plan's wait limit: the SM clock cycles (>= 1; default 2e9, about a second)
+ * a CTA waits for its own bulk copies before it records a timeout.  A diagnostic and
+ * a test hook: with a limit of a few cycles most waits run past it, and
+ * sketchssm_plan_check reports SKETCHSSM_ERR_TIMEOUT while the results stay complete.
+ * Applies to calls made after it; must not race with other calls on the plan.
+ */
+sketchssm_status sketchssm_plan_set_wait_limit(sketchssm_plan *plan, int64_t cycles);
 
 /* Free a plan and its device tables.  NULL is accepted.  Must not race with calls
  * that use the plan; device work already queued keeps its own copy of nothing, so

@@ -22,7 +22,7 @@ STATUS = {0: "SKETCHSSM_OK", 1: "SKETCHSSM_ERR_INVALID_ARG", 2: "SKETCHSSM_ERR_A
 
 # every symbol include/sketchssm.h declares
 EXPORTS = ("sketchssm_plan_create", "sketchssm_plan_query", "sketchssm_plan_check",
-           "sketchssm_plan_destroy", "sketchssm_flush", "sketchssm_decode", "sketchssm_dense_decode",
+           "sketchssm_plan_set_wait_limit", "sketchssm_plan_destroy", "sketchssm_flush", "sketchssm_decode", "sketchssm_dense_decode",
            "sketchssm_decode_static_scratch", "sketchssm_status_string", "sketchssm_last_error")
 
 
@@ -54,12 +54,13 @@ def load():
     lib.sketchssm_plan_create.argtypes = [ctypes.POINTER(Desc), P, P, ctypes.POINTER(P)]
     lib.sketchssm_plan_query.argtypes = [P, ctypes.POINTER(I64), P, P, I32, P, ctypes.POINTER(I32)]
     lib.sketchssm_plan_check.argtypes = [P, P]
+    lib.sketchssm_plan_set_wait_limit.argtypes = [P, I64]
     lib.sketchssm_plan_destroy.argtypes = [P]
     lib.sketchssm_flush.argtypes = [P, P, P, P, P, P, P, I32, P, P]
     lib.sketchssm_decode.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.sketchssm_dense_decode.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.sketchssm_decode_static_scratch.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
-    for f in EXPORTS[:8]:
+    for f in EXPORTS[:9]:
         getattr(lib, f).restype = ctypes.c_int
     lib.sketchssm_status_string.argtypes = [ctypes.c_int]
     lib.sketchssm_status_string.restype = ctypes.c_char_p
@@ -154,6 +155,11 @@ class Plan:
     def check(self, stream=None) -> None:
         """Synchronise and raise if a kernel recorded a timeout (sketchssm_plan_check)."""
         _check(load().sketchssm_plan_check(self.handle, _stream(stream)), "sketchssm_plan_check")
+
+    def set_wait_limit(self, cycles: int) -> None:
+        """Cycles a CTA waits for its own copies before it records a timeout
+        (sketchssm_plan_set_wait_limit; default 2e9)."""
+        _check(load().sketchssm_plan_set_wait_limit(self.handle, int(cycles)), "sketchssm_plan_set_wait_limit")
 
     def close(self) -> None:
         if getattr(self, "handle", None) is not None and self.handle.value:

@@ -397,13 +397,13 @@ combine_kernel(const DecodeArgs A)
         }
     }
     __syncthreads();
-    const bool ok = mbar_wait_bounded(bar, 0, A.wait_limit);
+    // a wait past the plan's limit is recorded (sketchssm_plan_check reports it) and then
+    // continued up to DEFAULT_WAIT_CYCLES; only a wait that outlasts both gives up
+    bool ok = mbar_wait_bounded(bar, 0, A.wait_limit);
     if (__syncthreads_or(!ok)) {
-        if (tid == 0) {
-            atomicOr(A.status, SK_STATUS_DECODE_TIMEOUT);
-            mbar_wait_bounded(bar, 0, A.wait_limit);  // a last chance for copies in flight
-        }
-        return;
+        if (tid == 0) atomicOr(A.status, SK_STATUS_DECODE_TIMEOUT);
+        ok = mbar_wait_bounded(bar, 0, DEFAULT_WAIT_CYCLES);
+        if (__syncthreads_or(!ok)) return;
     }
     const int V4 = V >> 2;
     for (int o = tid; o < nh * V4; o += blockDim.x) {

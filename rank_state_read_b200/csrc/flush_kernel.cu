@@ -126,10 +126,25 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, lo
                                               const volatile int *abort)
 {
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_poll(bar, parity, limit)) {
         if (*abort || clock64() - t0 > limit) return false;
     }
     return true;
+}
+
+// A wait past the plan's limit is recorded in the plan's status word (a timeout that
+// sketchssm_plan_check reports) and then continued, up to DEFAULT_WAIT_CYCLES more, for
+// the same phase, so that the copy protocol stays in order.  Only a wait that outlasts
+// both gives up: it sets the CTA's abort flag and returns false.
+__device__ __forceinline__ bool staged_wait(uint64_t *bar, uint32_t parity, const FlushArgs &A,
+                                            volatile int *abort)
+{
+    if (wait_or_abort(bar, parity, A.wait_limit, abort)) return true;
+    if (*abort) return false;
+    atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
+    if (wait_or_abort(bar, parity, DEFAULT_WAIT_CYCLES, abort)) return true;
+    *abort = 1;
+    return false;
 }
 
 // The producer warp requests an item's state slab and (n > 0) its buffered tokens,
@@ -342,7 +357,7 @@ flush_kernel(const FlushArgs A)
         bool ok = true;
         for (int j = 1; j <= cnt; ++j) {
             // every compute warp holds item j-1's slab and is done with item j-2
-            ok = wait_or_abort(empty, (uint32_t)((j - 1) & 1), A.wait_limit, abort);
+            ok = staged_wait(empty, (uint32_t)((j - 1) & 1), A, abort);
             if (!ok) break;
             if (pend_o) issue_omega(cur);  // item j-1's new basis rows
             pend_o = false;
@@ -361,8 +376,8 @@ flush_kernel(const FlushArgs A)
                 atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
             }
             // copies still in flight land before the CTA's shared memory is released
-            mbar_wait_bounded(full, last_full, A.wait_limit);
-            if (issued_o > 0) mbar_wait_bounded(obar, last_o, A.wait_limit);
+            mbar_wait_bounded(full, last_full, DEFAULT_WAIT_CYCLES);
+            if (issued_o > 0) mbar_wait_bounded(obar, last_o, DEFAULT_WAIT_CYCLES);
         }
         return;
     }
@@ -395,7 +410,7 @@ flush_kernel(const FlushArgs A)
             const float *T = Tb + (size_t)(j & 1) * cv.tfloats;
             const int r = cur.r;
             const bool need_o = new_group(cur);
-            ok = ok && wait_or_abort(full, (uint32_t)(j & 1), A.wait_limit, abort);
+            ok = ok && staged_wait(full, (uint32_t)(j & 1), A, abort);
             // the state in the accumulator layout: c[mt][nt][2 h + e] = state row
             // srow(mt, g, h), column col0 + 8 nt + 2 t + e
             float c[8][2][4];
@@ -507,7 +522,7 @@ flush_kernel(const FlushArgs A)
             // thread's 16 state rows, then a reduce-scatter over g (lane bits 2..4)
             // leaves sketch row m0 + g in lane 4 g + t
             if (need_o) {
-                ok = ok && wait_or_abort(obar, o_phase, A.wait_limit, abort);
+                ok = ok && staged_wait(obar, o_phase, A, abort);
                 o_phase ^= 1u;
             }
             if (r > 0 && ok) {
@@ -569,7 +584,7 @@ flush_kernel(const FlushArgs A)
         const int r = cur.r;
         const bool need_o = new_group(cur);
 
-        if (!wait_or_abort(full, (uint32_t)(j & 1), A.wait_limit, abort)) {
+        if (!staged_wait(full, (uint32_t)(j & 1), A, abort)) {
             if (lane == 0) {
                 *abort = 1;
                 atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
@@ -697,7 +712,7 @@ flush_kernel(const FlushArgs A)
         // by a reduce-scatter that leaves row m0 + ks in lane ks
         if (r > 0) {
             if (need_o) {
-                if (!wait_or_abort(obar, o_phase, A.wait_limit, abort)) {
+                if (!staged_wait(obar, o_phase, A, abort)) {
                     if (lane == 0) {
                         *abort = 1;
                         atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);

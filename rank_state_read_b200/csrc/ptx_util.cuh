@@ -53,12 +53,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// non-blocking test for the completion of phase `parity`
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Below this many cycles a wait limit is checked between non-blocking tests (try_wait
+// may suspend the thread until the phase completes, longer than a short limit).
+constexpr long long MBAR_SHORT_LIMIT = 65536;
+
+// one test of phase `parity`: non-blocking for a short limit, else possibly suspending
+__device__ __forceinline__ bool mbar_poll(uint64_t *bar, uint32_t parity, long long limit)
+{
+    return limit < MBAR_SHORT_LIMIT ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity);
+}
+
 // Wait for phase `parity` of the barrier for at most `limit` clock cycles.
 // Returns false if the limit ran out (the caller records the timeout).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, long long limit)
 {
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_poll(bar, parity, limit)) {
         if (clock64() - t0 > limit) return false;
     }
     return true;

@@ -361,9 +361,18 @@ sketchssm_status sketchssm_plan_check(const sketchssm_plan *p, sketchssm_stream 
         return cuda_fail(e, "cudaMemsetAsync(status)");
     if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream");
     if (flags & sk::SK_STATUS_DECODE_TIMEOUT)
-        return fail(SKETCHSSM_ERR_TIMEOUT, "a decode CTA gave up waiting for its bulk copies; its outputs are incomplete");
+        return fail(SKETCHSSM_ERR_TIMEOUT, "a decode CTA waited past the plan's limit for its bulk copies");
     if (flags & sk::SK_STATUS_FLUSH_TIMEOUT)
-        return fail(SKETCHSSM_ERR_TIMEOUT, "a flush CTA gave up waiting for its bulk copies; S and Y are incomplete");
+        return fail(SKETCHSSM_ERR_TIMEOUT, "a flush CTA waited past the plan's limit for its bulk copies");
+    return SKETCHSSM_OK;
+}
+
+sketchssm_status sketchssm_plan_set_wait_limit(sketchssm_plan *p, int64_t cycles)
+{
+    g_last_error.clear();
+    if (!p) return fail(SKETCHSSM_ERR_INVALID_ARG, "plan is NULL");
+    if (cycles < 1) return fail(SKETCHSSM_ERR_INVALID_ARG, "wait limit must be at least 1 cycle");
+    p->wait_limit = cycles;
     return SKETCHSSM_OK;
 }
 
