@@ -51,14 +51,14 @@ def test_short_wait_limit_is_reported_and_outputs_complete(cid):
         y_short = short.decode(pos, x["q"], x["k"], x["v"], x["a"], x["beta"]).clone()
         torch.cuda.synchronize()
         assert torch.equal(y_short, y_ref), pos
-    with pytest.raises(rs.SketchSSMError) as err:
-        short.plan.check()
-    assert err.value.status == 5  # SKETCHSSM_ERR_TIMEOUT
+    # a decode CTA whose copies landed before it waited records nothing; over the window
+    # cycle (the flush's producer and consumers wait on each other's items) the limit
+    # of one cycle is certainly overrun somewhere
     ref.flush(cfg.W)
     short.flush(cfg.W)
     with pytest.raises(rs.SketchSSMError) as err:
         short.plan.check()
-    assert err.value.status == 5
+    assert err.value.status == 5  # SKETCHSSM_ERR_TIMEOUT
     torch.cuda.synchronize()
     assert torch.equal(short.S, ref.S) and torch.equal(short.Y, ref.Y)
 
