@@ -38,6 +38,8 @@ def _load():
         lib.oracle_decode.argtypes = [ctypes.POINTER(_Dims), P, P, ctypes.c_int64,
                                       ctypes.c_int32, P, P, P, P, P, P, P, P, P, P, P, P,
                                       ctypes.c_int32, P]
+        lib.oracle_step.restype = None
+        lib.oracle_step.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -133,6 +135,22 @@ class OracleLayer:
                               _p(self.vbuf), _p(self.abuf), _p(self.bbuf), _p(self.Y),
                               _p(self.omega), _p(self.S), int(dense_all), _p(y))
         return y
+
+
+def standard_step(kind: str, S: np.ndarray, inp: dict, Hqk: int, lib=None) -> np.ndarray:
+    """The per-step recurrent decode (no buffer, no sketch): apply the step's token to
+    the fp64 state ``S`` [B][H][K][V] in place and return y = S^T q [B][H][V]."""
+    assert S.dtype == np.float64 and S.flags.c_contiguous
+    B, H, K, V = S.shape
+    q, k, v, a = (_f64(inp[x]) for x in ("q", "k", "v", "a"))
+    beta = None if inp.get("beta") is None else _f64(inp["beta"])
+    assert q.shape == (B, Hqk, K) and k.shape == q.shape and v.shape == (B, H, V)
+    if kind != "mamba2":
+        assert beta is not None and beta.shape == (B, H)
+    dims = _Dims(KIND_ID[kind], B, H, Hqk, K, V, 1, 1, 1)
+    y = np.empty((B, H, V))
+    (lib or _load()).oracle_step(ctypes.byref(dims), _p(S), _p(q), _p(k), _p(v), _p(a), _p(beta), _p(y))
+    return y
 
 
 def trajectory(layer: OracleLayer, inputs: Iterable[dict], *, dense_all: bool = False,

@@ -223,6 +223,51 @@ void oracle_decode(const oracle_dims *d, const int32_t *rank, const int32_t *off
     }
 }
 
+/* ------------------------------------------------------------------ standard step
+ * The per-step recurrent decode the paper measures its speedup against [ABS: standard
+ * decoding reads and updates the full state for every token]: for every (b, h), apply
+ * the step's token to the state, S <- M S + beta k v^T (the transition table above;
+ * Mamba-2 beta = 1), then read it, y = S^T q (read after the update, as in the
+ * decode).  No buffer, no sketch.  Inputs of one step: q, k [B][Hqk][K],
+ * v [B][H][V], a [B][H] (KDA [B][H][K]), beta [B][H] (unused for Mamba-2). */
+void oracle_step(const oracle_dims *d, double *S, const double *q, const double *k, const double *v,
+                 const double *a, const double *beta, double *y)
+{
+    const int64_t K = d->K, V = d->V;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < d->B; ++b) {
+        for (int64_t h = 0; h < d->H; ++h) {
+            const int64_t bh = b * d->H + h;
+            const int64_t qh = (h * d->Hqk) / d->H;
+            double *Sh = S + bh * K * V;
+            const double *kt = k + (b * d->Hqk + qh) * K;
+            const double *qt = q + (b * d->Hqk + qh) * K;
+            const double *vt = v + bh * V;
+            if (d->kind == ORACLE_MAMBA2) {
+                const double at = a[bh];
+                for (int64_t kk = 0; kk < K; ++kk)
+                    for (int64_t j = 0; j < V; ++j) Sh[kk * V + j] = at * Sh[kk * V + j] + kt[kk] * vt[j];
+            } else {
+                const double bt = beta[bh];
+                for (int64_t j = 0; j < V; ++j) {
+                    double e = 0.0; /* (k^T S)_j, taken before the update */
+                    for (int64_t kk = 0; kk < K; ++kk) e += kt[kk] * Sh[kk * V + j];
+                    for (int64_t kk = 0; kk < K; ++kk) {
+                        const double at = (d->kind == ORACLE_KDA) ? a[bh * K + kk] : a[bh];
+                        Sh[kk * V + j] = at * (Sh[kk * V + j] - bt * kt[kk] * e) + bt * kt[kk] * vt[j];
+                    }
+                }
+            }
+            double *yo = y + bh * V;
+            for (int64_t j = 0; j < V; ++j) {
+                double s = 0.0;
+                for (int64_t kk = 0; kk < K; ++kk) s += Sh[kk * V + j] * qt[kk];
+                yo[j] = s;
+            }
+        }
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

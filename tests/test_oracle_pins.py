@@ -331,3 +331,64 @@ def test_mutations_are_caught(name, old, new, kind, tmp_path):
     cfg = tiny_cfg(kind, Hqk=2 if kind == "mamba2" else None)
     rank = np.array([1, DENSE, 2, 3], np.int32)
     assert check_against_brute(cfg, rank, T=2 * cfg.W + 3, lib=lib) > 1e-6
+
+
+# --------------------------------------------------------------------------- standard step
+
+def check_step_against_brute(cfg, T, lib=None):
+    """The per-step recurrent decode (oracle.standard_step) against the token-by-token
+    definition with explicit transition matrices (brute.run_row's exact read)."""
+    rows = list(range(cfg.B))
+    S = np.ascontiguousarray(synth.init_state(cfg, rows), dtype=np.float64)
+    S0 = S.copy()
+    steps = [synth.step_inputs(cfg, t, rows) for t in range(T)]
+    rank = np.full(cfg.H, DENSE, np.int32)
+    bf = [brute.run_row(cfg.kind, S0[b], [{x: (None if s[x] is None else s[x][b]) for x in s} for s in steps],
+                        rank, synth.basis_fp64(cfg), cfg.G, cfg.Hqk, cfg.W) for b in rows]
+    worst = 0.0
+    for t, inp in enumerate(steps):
+        y = oracle.standard_step(cfg.kind, S, inp, cfg.Hqk, lib=lib)
+        worst = max(worst, rel(y, np.stack([bf[b]["y_exact"][t] for b in rows])))
+    return worst
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+@pytest.mark.parametrize("shared_qk", [False, True])
+def test_standard_step_brute_force(kind, shared_qk):
+    """One token applied to the full state and read after the update, every step: equal
+    to the explicit-matrix definition over two windows plus a ragged tail."""
+    cfg = tiny_cfg(kind, Hqk=2 if shared_qk else None)
+    assert check_step_against_brute(cfg, T=2 * cfg.W + 3) < 1e-12
+
+
+def test_standard_step_full_head_shape():
+    cfg = tiny_cfg("kda", H=2, G=1, K=128, V=128, W=16, B=1, seed=9)
+    assert check_step_against_brute(cfg, T=5) < 1e-11
+
+
+STEP_MUTATIONS = [
+    ("step drops the decay",
+     "Sh[kk * V + j] = at * Sh[kk * V + j] + kt[kk] * vt[j];",
+     "Sh[kk * V + j] = Sh[kk * V + j] + kt[kk] * vt[j];", "mamba2"),
+    ("step erase sign",
+     "at * (Sh[kk * V + j] - bt * kt[kk] * e)",
+     "at * (Sh[kk * V + j] + bt * kt[kk] * e)", "gdn"),
+    ("step erase outside the decay",
+     "at * (Sh[kk * V + j] - bt * kt[kk] * e)",
+     "(at * Sh[kk * V + j] - bt * kt[kk] * e)", "kda"),
+    ("step reads with the key",
+     "s += Sh[kk * V + j] * qt[kk];",
+     "s += Sh[kk * V + j] * kt[kk];", "gdn"),
+]
+
+
+@pytest.mark.parametrize("name,old,new,kind", STEP_MUTATIONS, ids=[m[0] for m in STEP_MUTATIONS])
+def test_step_mutations_are_caught(name, old, new, kind, tmp_path):
+    src = open(obuild.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique: {old!r}"
+    mutated = tmp_path / "mut.c"
+    mutated.write_text(src.replace(old, new))
+    out = str(tmp_path / "libmut.so")
+    obuild.build(force=True, src=str(mutated), out=out)
+    lib = oracle.load_library(out)
+    assert check_step_against_brute(tiny_cfg(kind, Hqk=2 if kind == "mamba2" else None), T=7, lib=lib) > 1e-6
