@@ -75,6 +75,15 @@ def dense_decode_bytes(cfg, pos: int) -> int:
     return cfg.B * row
 
 
+def step_bytes(cfg) -> int:
+    """Algorithmic HBM bytes of one standard per-step decode launch: the state read and
+    written, plus q, k (per q/k head), v, a, beta read and y written, per batch row."""
+    da = cfg.K if cfg.kda else 1
+    per_row = (2 * cfg.H * cfg.K * cfg.V + 2 * cfg.Hqk * cfg.K + 2 * cfg.H * cfg.V + cfg.H * da
+               + (cfg.H if cfg.has_beta else 0))
+    return 4 * cfg.B * per_row
+
+
 def flush_bytes(cfg, rank, n: int) -> int:
     """One flush of n buffered tokens: the state read and written once, the n tokens
     read, the sketch written; plus the basis rows once per launch."""
@@ -298,7 +307,8 @@ def run_ours(args, cfg) -> None:
     ms = t_start.elapsed_time(t_end)
     dec = [(p, a.elapsed_time(b)) for p, a, b in ev["decode"]]
     fl = [b_.elapsed_time(c_) for _, b_, c_ in ev["flush"]]
-    launches = len(ev["decode"]) + len(ev["flush"])
+    # every decode call is two launches (the products kernel and the combine kernel)
+    launches = 2 * len(ev["decode"]) + len(ev["flush"])
 
     # ---- dense-read baseline decode (same positions, same replicas)
     kd = max(1, min(args.steps, 10))
@@ -310,6 +320,23 @@ def run_ours(args, cfg) -> None:
     dd = [(p, a.elapsed_time(b)) for p, a, b in evd["decode"]]
     for lay in layers:   # the dense-read cycles left W tokens buffered: apply them
         lay.flush(cfg.W)
+
+    # ---- standard per-step decode (full state read and updated every token), the
+    # baseline the pages' speedups are quoted against: same replicas, same tokens
+    st_ev = []
+    barrier()
+    for _ in range(kd):
+        for p in range(cfg.W):
+            for l, lay in enumerate(layers):
+                x = inputs[l][p]
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                lay.standard_step(x["q"], x["k"], x["v"], x["a"], x["beta"])
+                e1 = torch.cuda.Event(enable_timing=True)
+                e1.record(stream)
+                st_ev.append((e0, e1))
+    barrier()
+    st = [a.elapsed_time(b) for a, b in st_ev]
 
     # ---- end to end through the C ABI: inputs from pinned host memory, y back to host
     host_in = [{k: (None if v is None else v.cpu().pin_memory()) for k, v in inputs[0][p].items()}
@@ -358,6 +385,8 @@ def run_ours(args, cfg) -> None:
     mean_dec_us = 1e3 * dec_ms / len(dec)
     mean_fl_us = 1e3 * fl_ms / len(fl)
     mean_dd_us = 1e3 * dd_ms / len(dd)
+    mean_st_us = 1e3 * sum(st) / len(st)
+    st_gbs = step_bytes(cfg) / (mean_st_us * 1e-6) / 1e9
 
     def roof(kernel, achieved, nbytes_per_launch):
         tr = kernel_traffic(kernel)
@@ -394,6 +423,9 @@ def run_ours(args, cfg) -> None:
                        "decode_only_tok_s": round(cfg.B * world / (mean_dd_us / 1e6), 1)},
         "speedup_vs_dense_read": round(mean_dd_us / mean_dec_us, 3),
         "traffic_ratio_dense_over_sketch": round(dd_bytes / len(dd) / (dec_bytes / len(dec)), 3),
+        "standard_step": {"step_us": round(mean_st_us, 2), "hbm_gbs": round(st_gbs, 1),
+                          "frac": round(st_gbs / peak, 4), "tok_s": round(cfg.B / (mean_st_us * 1e-6), 1)},
+        "speedup_vs_standard_step": round(cfg.W * mean_st_us / (cfg.W * mean_dec_us + mean_fl_us), 3),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d // ke,
                 "d2h_bytes_per_step": d2h // ke,
                 "note": "pinned host inputs copied in and y copied out around every decode call"},

@@ -236,6 +236,21 @@ sketchssm_status sketchssm_decode_static_scratch(const sketchssm_plan *plan, int
                                                  const float *S, float *y,
                                                  sketchssm_stream stream);
 
+/*
+ * Standard per-step recurrent decode: the baseline the paper compares against (paper
+ * abstract: standard decoding reads and updates the full state for every token).  For
+ * every (b, h) apply the step's token to S in place, S <- M S + beta k v^T, and write
+ * y[b][h] = S^T q, read after the update.  No buffer or sketch is read or written; the
+ * plan supplies only the shape (its rank table is not used).  Tensors and layouts as in
+ * the general conventions (q, k [B][Hqk][K], v [B][H][V], a [B][H] or KDA [B][H][K],
+ * beta [B][H] or NULL for Mamba-2, S [B][H][K][V], y [B][H][V]).  A state driven only by
+ * this call matches the state of the sketch path's decode / flush protocol after every
+ * flush (the same recurrence), and y equals the exact read at every step.
+ */
+sketchssm_status sketchssm_step(const sketchssm_plan *plan, const float *q, const float *k,
+                                const float *v, const float *a, const float *beta, float *S,
+                                float *y, sketchssm_stream stream);
+
 /* Static text of a status code. */
 const char *sketchssm_status_string(sketchssm_status status);
 

@@ -20,5 +20,6 @@ from ._binding import (  # noqa: F401
     sketchssm_flush,
     sketchssm_plan_create,
     sketchssm_plan_destroy,
+    sketchssm_step,
 )
 from .layer import SketchLayer  # noqa: F401

@@ -23,7 +23,8 @@ STATUS = {0: "SKETCHSSM_OK", 1: "SKETCHSSM_ERR_INVALID_ARG", 2: "SKETCHSSM_ERR_A
 # every symbol include/sketchssm.h declares
 EXPORTS = ("sketchssm_plan_create", "sketchssm_plan_query", "sketchssm_plan_check",
            "sketchssm_plan_set_wait_limit", "sketchssm_plan_destroy", "sketchssm_flush", "sketchssm_decode", "sketchssm_dense_decode",
-           "sketchssm_decode_static_scratch", "sketchssm_status_string", "sketchssm_last_error")
+           "sketchssm_decode_static_scratch", "sketchssm_step", "sketchssm_status_string",
+           "sketchssm_last_error")
 
 
 class SketchSSMError(RuntimeError):
@@ -60,7 +61,8 @@ def load():
     lib.sketchssm_decode.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.sketchssm_dense_decode.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.sketchssm_decode_static_scratch.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
-    for f in EXPORTS[:9]:
+    lib.sketchssm_step.argtypes = [P, P, P, P, P, P, P, P, P]
+    for f in EXPORTS[:10]:
         getattr(lib, f).restype = ctypes.c_int
     lib.sketchssm_status_string.argtypes = [ctypes.c_int]
     lib.sketchssm_status_string.restype = ctypes.c_char_p
@@ -221,3 +223,12 @@ def sketchssm_decode_static_scratch(plan: Plan, pos: int, q, k, v, a, beta, kbuf
         _ptr(vbuf, "vbuf", n("vbuf")), _ptr(abuf, "abuf", n("abuf")), _ptr(bbuf, "bbuf", n("bbuf")),
         _ptr(Y, "Y", n("Y")), _ptr(omega, "omega", n("omega")), _ptr(S, "S", n("S")),
         _ptr(y, "y", n("y")), _stream(stream)), "sketchssm_decode_static_scratch")
+
+
+def sketchssm_step(plan: Plan, q, k, v, a, beta, S, y, stream=None) -> None:
+    """The standard per-step decode (sketchssm_step): S updated in place, y = S^T q."""
+    n = plan.numel
+    _check(load().sketchssm_step(
+        plan.handle, _ptr(q, "q", n("q")), _ptr(k, "k", n("k")), _ptr(v, "v", n("v")), _ptr(a, "a", n("a")),
+        _ptr(beta, "beta", n("beta")), _ptr(S, "S", n("S")), _ptr(y, "y", n("y")), _stream(stream)),
+        "sketchssm_step")

@@ -18,6 +18,7 @@ constexpr int MAX_V = 256;       // value dim
 // bits of the plan's device status word
 constexpr int SK_STATUS_DECODE_TIMEOUT = 1;
 constexpr int SK_STATUS_FLUSH_TIMEOUT = 2;
+constexpr int SK_STATUS_STEP_TIMEOUT = 4;
 
 // default bound of a kernel's wait on its own bulk copies (clock cycles, ~1 s)
 constexpr long long DEFAULT_WAIT_CYCLES = 2000000000LL;
@@ -79,6 +80,18 @@ int coef_rows(int cap, int W);
 int dots_row(int W, int cap);
 size_t decode_smem_bytes(const DecodeArgs &a);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+// Arguments of one standard per-step decode launch.
+struct StepArgs {
+    int kind, B, H, Hqk, V, hpq;
+    int VS;  // column slab of one CTA
+    long long wait_limit;
+    int *status;
+    const float *q, *k, *v, *a, *beta;
+    float *S, *y;
+};
+int step_slab(int V);
+cudaError_t launch_step(const StepArgs &a, cudaStream_t stream);
 
 int flush_slab(int V);
 size_t flush_smem_bytes(int kind, int V, int W, int rcap);

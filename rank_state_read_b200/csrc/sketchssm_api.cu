@@ -362,6 +362,8 @@ sketchssm_status sketchssm_plan_check(const sketchssm_plan *p, sketchssm_stream 
     if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream");
     if (flags & sk::SK_STATUS_DECODE_TIMEOUT)
         return fail(SKETCHSSM_ERR_TIMEOUT, "a decode CTA waited past the plan's limit for its bulk copies");
+    if (flags & sk::SK_STATUS_STEP_TIMEOUT)
+        return fail(SKETCHSSM_ERR_TIMEOUT, "a standard-step CTA waited past the plan's limit for its bulk copies");
     if (flags & sk::SK_STATUS_FLUSH_TIMEOUT)
         return fail(SKETCHSSM_ERR_TIMEOUT, "a flush CTA waited past the plan's limit for its bulk copies");
     return SKETCHSSM_OK;
@@ -567,5 +569,45 @@ extern "C" sketchssm_status sketchssm_decode_static_scratch(const sketchssm_plan
     A.scratch = scratch;
     cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch (static scratch)");
+    return SKETCHSSM_OK;
+}
+
+extern "C" sketchssm_status sketchssm_step(const sketchssm_plan *p, const float *q, const float *k,
+                                           const float *v, const float *a, const float *beta, float *S,
+                                           float *y, sketchssm_stream stream)
+{
+    g_last_error.clear();
+    sketchssm_status s = check_plan(p);
+    if (s != SKETCHSSM_OK) return s;
+    const sketchssm_desc &d = p->d;
+    const long long B = d.batch, H = d.heads, Q = d.qk_heads, K = d.key_dim, V = d.value_dim;
+    const long long da = d.kind == SKETCHSSM_KDA ? K : 1;
+    const bool mamba = d.kind == SKETCHSSM_MAMBA2;
+    CHECK_T(q, fbytes(B, Q, K), "q", false);
+    CHECK_T(k, fbytes(B, Q, K), "k", false);
+    CHECK_T(v, fbytes(B, H, V), "v", false);
+    CHECK_T(a, fbytes(B, H, da), "a", false);
+    CHECK_T(beta, mamba ? 0 : fbytes(B, H), "beta", mamba);
+    CHECK_T(S, fbytes(B, H, K, V), "S", false);
+    CHECK_T(y, fbytes(B, H, V), "y", false);
+    sk::StepArgs A;
+    A.kind = d.kind;
+    A.B = d.batch;
+    A.H = d.heads;
+    A.Hqk = d.qk_heads;
+    A.V = d.value_dim;
+    A.hpq = p->hpq;
+    A.VS = sk::step_slab(d.value_dim);
+    A.wait_limit = p->wait_limit;
+    A.status = p->d_status;
+    A.q = q;
+    A.k = k;
+    A.v = v;
+    A.a = a;
+    A.beta = beta;
+    A.S = S;
+    A.y = y;
+    cudaError_t e = sk::launch_step(A, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "standard step kernel launch");
     return SKETCHSSM_OK;
 }

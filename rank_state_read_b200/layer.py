@@ -10,7 +10,7 @@ from typing import Optional, Sequence
 import numpy as np
 import torch
 
-from ._binding import Plan, sketchssm_decode, sketchssm_dense_decode, sketchssm_flush
+from ._binding import Plan, sketchssm_decode, sketchssm_dense_decode, sketchssm_flush, sketchssm_step
 
 
 def _dev(x, device) -> torch.Tensor:
@@ -60,6 +60,13 @@ class SketchLayer:
         y = self.y if out is None else out
         sketchssm_dense_decode(self.plan, pos, q, k, v, a, beta, self.kbuf, self.vbuf, self.abuf,
                                self.bbuf, self.S, y, stream)
+        return y
+
+    def standard_step(self, q, k, v, a, beta: Optional[torch.Tensor] = None, out=None,
+                      stream=None) -> torch.Tensor:
+        """The per-step recurrent decode (no buffer): S updated in place, y = S^T q."""
+        y = self.y if out is None else out
+        sketchssm_step(self.plan, q, k, v, a, beta, self.S, y, stream)
         return y
 
     def close(self) -> None:
