@@ -237,6 +237,35 @@ sketchssm_status sketchssm_decode_static_scratch(const sketchssm_plan *plan, int
                                                  sketchssm_stream stream);
 
 /*
+ * Per-sequence positions (continuous batching): sketchssm_decode with a position per
+ * batch row.  pos is a device array [B] of int32 (16-byte aligned); row b appends its
+ * token at its own buffer slot pos[b] and replays pos[b] + 1 tokens.  Rows move through
+ * their windows independently; sketchssm_flush_rows applies each row's tokens.  A
+ * position outside [0, W) cannot be seen on the host: the kernels leave that row
+ * unchanged (no y, no append) and sketchssm_plan_check reports SKETCHSSM_ERR_INVALID_ARG.
+ * Everything else as sketchssm_decode.  Source: the serving setting of the sketchssm
+ * PyPI page (vLLM batches sequences at different positions).
+ */
+sketchssm_status sketchssm_decode_rows(const sketchssm_plan *plan, const int32_t *pos, const float *q,
+                                       const float *k, const float *v, const float *a,
+                                       const float *beta, float *kbuf, float *vbuf, float *abuf,
+                                       float *bbuf, const float *Y, const float *omega,
+                                       const float *S, float *y, sketchssm_stream stream);
+
+/*
+ * Per-row flush: sketchssm_flush with a token count per batch row.  n_tokens is a device
+ * array [B] of int32 in [0, W] (16-byte aligned); row b applies its buffer slots
+ * 0 .. n_tokens[b]-1 to its state and re-forms its sketch rows.  A row with 0 tokens is
+ * left untouched (its state and sketch keep their values; the initial sketch of a fresh
+ * state is formed with sketchssm_flush(n_tokens = 0)).  A count outside [0, W] leaves
+ * the row untouched and is reported by sketchssm_plan_check as SKETCHSSM_ERR_INVALID_ARG.
+ */
+sketchssm_status sketchssm_flush_rows(const sketchssm_plan *plan, float *S, const float *omega,
+                                      const float *kbuf, const float *vbuf, const float *abuf,
+                                      const float *bbuf, const int32_t *n_tokens, float *Y,
+                                      sketchssm_stream stream);
+
+/*
  * Standard per-step recurrent decode: the baseline the paper compares against (paper
  * abstract: standard decoding reads and updates the full state for every token).  For
  * every (b, h) apply the step's token to S in place, S <- M S + beta k v^T, and write

@@ -15,9 +15,11 @@ from ._binding import (  # noqa: F401
     SketchSSMError,
     load,
     sketchssm_decode,
+    sketchssm_decode_rows,
     sketchssm_decode_static_scratch,
     sketchssm_dense_decode,
     sketchssm_flush,
+    sketchssm_flush_rows,
     sketchssm_plan_create,
     sketchssm_plan_destroy,
     sketchssm_step,

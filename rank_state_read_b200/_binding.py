@@ -23,8 +23,8 @@ STATUS = {0: "SKETCHSSM_OK", 1: "SKETCHSSM_ERR_INVALID_ARG", 2: "SKETCHSSM_ERR_A
 # every symbol include/sketchssm.h declares
 EXPORTS = ("sketchssm_plan_create", "sketchssm_plan_query", "sketchssm_plan_check",
            "sketchssm_plan_set_wait_limit", "sketchssm_plan_destroy", "sketchssm_flush", "sketchssm_decode", "sketchssm_dense_decode",
-           "sketchssm_decode_static_scratch", "sketchssm_step", "sketchssm_status_string",
-           "sketchssm_last_error")
+           "sketchssm_decode_static_scratch", "sketchssm_step", "sketchssm_decode_rows",
+           "sketchssm_flush_rows", "sketchssm_status_string", "sketchssm_last_error")
 
 
 class SketchSSMError(RuntimeError):
@@ -62,7 +62,9 @@ def load():
     lib.sketchssm_dense_decode.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.sketchssm_decode_static_scratch.argtypes = [P, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.sketchssm_step.argtypes = [P, P, P, P, P, P, P, P, P]
-    for f in EXPORTS[:10]:
+    lib.sketchssm_decode_rows.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
+    lib.sketchssm_flush_rows.argtypes = [P, P, P, P, P, P, P, P, P, P]
+    for f in EXPORTS[:12]:
         getattr(lib, f).restype = ctypes.c_int
     lib.sketchssm_status_string.argtypes = [ctypes.c_int]
     lib.sketchssm_status_string.restype = ctypes.c_char_p
@@ -232,3 +234,33 @@ def sketchssm_step(plan: Plan, q, k, v, a, beta, S, y, stream=None) -> None:
         plan.handle, _ptr(q, "q", n("q")), _ptr(k, "k", n("k")), _ptr(v, "v", n("v")), _ptr(a, "a", n("a")),
         _ptr(beta, "beta", n("beta")), _ptr(S, "S", n("S")), _ptr(y, "y", n("y")), _stream(stream)),
         "sketchssm_step")
+
+
+def _rows(t, name: str, B: int):
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous int32 CUDA tensor")
+    if t.numel() != B:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {B}")
+    return t.data_ptr()
+
+
+def sketchssm_decode_rows(plan: Plan, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, Y, omega, S, y,
+                          stream=None) -> None:
+    """sketchssm_decode with a buffer position per batch row (pos: int32 [B] on the device)."""
+    n = plan.numel
+    _check(load().sketchssm_decode_rows(
+        plan.handle, _rows(pos, "pos", plan.desc.batch), _ptr(q, "q", n("q")), _ptr(k, "k", n("k")),
+        _ptr(v, "v", n("v")), _ptr(a, "a", n("a")), _ptr(beta, "beta", n("beta")), _ptr(kbuf, "kbuf", n("kbuf")),
+        _ptr(vbuf, "vbuf", n("vbuf")), _ptr(abuf, "abuf", n("abuf")), _ptr(bbuf, "bbuf", n("bbuf")),
+        _ptr(Y, "Y", n("Y")), _ptr(omega, "omega", n("omega")), _ptr(S, "S", n("S")), _ptr(y, "y", n("y")),
+        _stream(stream)), "sketchssm_decode_rows")
+
+
+def sketchssm_flush_rows(plan: Plan, S, omega, kbuf, vbuf, abuf, bbuf, n_tokens, Y, stream=None) -> None:
+    """sketchssm_flush with a token count per batch row (n_tokens: int32 [B] on the device)."""
+    n = plan.numel
+    _check(load().sketchssm_flush_rows(
+        plan.handle, _ptr(S, "S", n("S")), _ptr(omega, "omega", n("omega")), _ptr(kbuf, "kbuf", n("kbuf")),
+        _ptr(vbuf, "vbuf", n("vbuf")), _ptr(abuf, "abuf", n("abuf")), _ptr(bbuf, "bbuf", n("bbuf")),
+        _rows(n_tokens, "n_tokens", plan.desc.batch), _ptr(Y, "Y", n("Y")), _stream(stream)),
+        "sketchssm_flush_rows")

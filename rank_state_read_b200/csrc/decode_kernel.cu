@@ -50,6 +50,20 @@ constexpr int COEF_THREADS = 128;
 
 __host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
 
+// Buffer position of batch row b: the call's pos, or the row's own (per-row positions).
+// A position outside [0, W) is recorded (sketchssm_plan_check reports it) and -1 is
+// returned: the caller then leaves the row alone.
+__device__ __forceinline__ int row_position(const DecodeArgs &A, int b)
+{
+    if (!A.row_pos) return A.pos;
+    const int p = __ldg(A.row_pos + b);
+    if (p < 0 || p >= A.W) {
+        atomicOr(A.status, SK_STATUS_BAD_ROW);
+        return -1;
+    }
+    return p;
+}
+
 // ============================================================================ query-side products
 
 constexpr int CM_THREADS = 256;
@@ -95,10 +109,16 @@ dots_kernel_mamba2(const DecodeArgs A)
     extern __shared__ __align__(128) unsigned char cms[];
     pdl_launch_dependents();  // the combine may start staging its rows now
     const int tid = threadIdx.x;
-    const int W = A.W, pos = A.pos, n = pos + 1, hpq = A.hpq, cap = A.cap, dr = A.dots_row;
+    const int W = A.W, hpq = A.hpq, cap = A.cap, dr = A.dots_row;
     const int rows = A.cm_rows;
     const int q = blockIdx.x, b0 = blockIdx.y * rows;
     const int nb = min(rows, A.B - b0);
+    // buffer position of each of the CTA's rows (-1: a bad per-row position, row skipped)
+    __shared__ int rpos[CM_MAXROWS];
+    if (tid < nb) rpos[tid] = row_position(A, b0 + tid);
+    __syncthreads();
+    int nmax = 0;  // key slots in use in any of the rows (all rows alike: pos + 1)
+    for (int bl = 0; bl < nb; ++bl) nmax = max(nmax, rpos[bl] + 1);
     const int g = (q * hpq) / A.Hg;
     const CmCarve cv = cm_carve(cap, W, rows);
     float *om = reinterpret_cast<float *>(cms + cv.om);  // [rq][OPAD]
@@ -115,8 +135,9 @@ dots_kernel_mamba2(const DecodeArgs A)
         const int bl = x >> 5, c = x & 31;
         cp_async16(qs + bl * OPAD + c * 4, A.q + ((long long)(b0 + bl) * A.Hqk + q) * KDIM + c * 4);
     }
-    for (int x = tid; x < nb * n * (KDIM / 4); x += CM_THREADS) {
-        const int c = x & 31, r = x >> 5, bl = r / n, i = r - bl * n;
+    for (int x = tid; x < nb * nmax * (KDIM / 4); x += CM_THREADS) {
+        const int c = x & 31, r = x >> 5, bl = r / nmax, i = r - bl * nmax, pos = rpos[bl];
+        if (i > pos) continue;
         const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
         cp_async16(ks + bl * cv.kblock + i * OPAD + c * 4,
                    (i == pos ? A.k + qrow * KDIM : A.kbuf + (qrow * W + i) * KDIM) + c * 4);
@@ -125,14 +146,17 @@ dots_kernel_mamba2(const DecodeArgs A)
     // unused entries of the rows: 0
     for (int x = tid; x < nb * dr; x += CM_THREADS) {
         const int bl = x / dr, e = x - bl * dr;
-        if ((e >= n && e < W) || e >= W + rq) A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + e] = 0.f;
+        if (rpos[bl] < 0) continue;
+        if ((e > rpos[bl] && e < W) || e >= W + rq) A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + e] = 0.f;
     }
     cp_async_wait<0>();
     __syncthreads();
 
-    for (int t = tid; t < (n + rq) * nb; t += CM_THREADS) {
+    // task (row rr, batch row): rr < nmax a key slot, else basis row rr - nmax
+    for (int t = tid; t < (nmax + rq) * nb; t += CM_THREADS) {
         const int rr = t / nb, bl = t - rr * nb;
-        const float *row = rr < n ? ks + bl * cv.kblock + rr * OPAD : om + (size_t)(rr - n) * OPAD;
+        if (rr < nmax && rr > rpos[bl]) continue;
+        const float *row = rr < nmax ? ks + bl * cv.kblock + rr * OPAD : om + (size_t)(rr - nmax) * OPAD;
         const float *qb = qs + (size_t)bl * OPAD;
         float4 acc = zero4();
 #pragma unroll 8
@@ -143,12 +167,13 @@ dots_kernel_mamba2(const DecodeArgs A)
             acc.z = fmaf(o.z, v.z, acc.z);
             acc.w = fmaf(o.w, v.w, acc.w);
         }
-        A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + (rr < n ? rr : W + rr - n)] =
+        A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + (rr < nmax ? rr : W + rr - nmax)] =
             (acc.x + acc.y) + (acc.z + acc.w);
     }
     // the step's key goes to buffer slot pos (from the stage)
     for (int x = tid; x < nb * (KDIM / 4); x += CM_THREADS) {
-        const int bl = x >> 5, c = x & 31;
+        const int bl = x >> 5, c = x & 31, pos = rpos[bl];
+        if (pos < 0) continue;
         const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
         st4(A.kbuf + (qrow * W + pos) * KDIM + c * 4, lds4(ks + bl * cv.kblock + pos * OPAD + c * 4));
     }
@@ -162,8 +187,10 @@ coef_kernel_delta(const DecodeArgs A)
     pdl_launch_dependents();  // the combine may start staging its rows now
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int h = blockIdx.x * (COEF_THREADS / 32) + warp, b = blockIdx.y;
-    const int H = A.H, W = A.W, pos = A.pos, n = pos + 1, hpq = A.hpq;
-    if (h >= H) return;
+    if (h >= A.H) return;
+    const int pos = row_position(A, b);
+    if (pos < 0) return;
+    const int H = A.H, W = A.W, n = pos + 1, hpq = A.hpq;
     const int qk = h / hpq, g = h / A.Hg;
     const long long bh = (long long)b * H + h;
     const long long qrow = (long long)b * A.Hqk + qk;
@@ -302,7 +329,15 @@ combine_kernel(const DecodeArgs A)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.y;
-    const int H = A.H, V = A.V, W = A.W, pos = A.pos, n = pos + 1, hpq = A.hpq, dr = A.dots_row;
+    const int pos = row_position(A, b);
+    if (pos < 0) return;
+    const int H = A.H, V = A.V, W = A.W, n = pos + 1, hpq = A.hpq, dr = A.dots_row;
+    // per-row positions: this row's work list (the launch covers the longest list)
+    const int *rec_list = A.rec;
+    if (A.row_pos && !A.dense_all) {
+        if ((int)blockIdx.x >= __ldg(A.counts + 2 + n)) return;
+        rec_list = A.rec + (size_t)(n - 1) * (H + A.G) * 8;
+    }
     // the item's record: {entry, span, member mask, rows R, off[h_first], coff[h_first], coef floats, h_first}
     int R, yrow0, c0, cfl, h_first;
     unsigned mask;
@@ -316,8 +351,8 @@ combine_kernel(const DecodeArgs A)
         c0 = h_first * A.coef_dense_block;
         cfl = A.coef_dense_block;
     } else {
-        const int4 r0 = __ldg(reinterpret_cast<const int4 *>(A.rec) + 2 * blockIdx.x);
-        const int4 r1 = __ldg(reinterpret_cast<const int4 *>(A.rec) + 2 * blockIdx.x + 1);
+        const int4 r0 = __ldg(reinterpret_cast<const int4 *>(rec_list) + 2 * blockIdx.x);
+        const int4 r1 = __ldg(reinterpret_cast<const int4 *>(rec_list) + 2 * blockIdx.x + 1);
         dense = r0.x < 0;
         mask = (unsigned)r0.z;
         R = r0.w;

@@ -92,10 +92,27 @@ __host__ __device__ inline FlushCarve flush_carve(int kind, int VS, int W, int r
     return c;
 }
 
+// Tokens a batch row applies: the call's n, or the row's own count (per-row counts).
+// A count outside [0, W] is recorded (sketchssm_plan_check reports it) and the row is
+// left alone (0).
+__device__ __forceinline__ int row_tokens(const FlushArgs &A, int b)
+{
+    if (!A.row_n) return A.n;
+    const int n = __ldg(A.row_n + b);
+    if (n < 0 || n > A.W) {
+        atomicOr(A.status, SK_STATUS_BAD_ROW);
+        return 0;
+    }
+    return n;
+}
+
 // (b, h, slab) of consecutive items, advanced without divisions; the head's rank and
-// sketch-row offset are loaded when the cursor moves (one item before they are used)
+// sketch-row offset are loaded when the cursor moves (one item before they are used).
+// n: the row's tokens; proj: whether the item re-forms its sketch rows (a sketch head,
+// and with per-row counts only a row that applies tokens)
 struct Cursor {
-    int b, h, slab, r, off;
+    int b, h, slab, r, off, n;
+    bool proj;
     __device__ void init(const FlushArgs &A, long long item, int nslab)
     {
         const long long bh = item / nslab;
@@ -104,6 +121,8 @@ struct Cursor {
         h = (int)(bh - (long long)b * A.H);
         r = __ldg(A.rank + h);
         off = __ldg(A.off + h);
+        n = row_tokens(A, b);
+        proj = r > 0 && (!A.row_n || n > 0);
     }
     __device__ void next(const FlushArgs &A, int nslab)
     {
@@ -112,9 +131,11 @@ struct Cursor {
             if (++h == A.H) {
                 h = 0;
                 ++b;
+                n = row_tokens(A, b);
             }
             r = __ldg(A.rank + h);
             off = __ldg(A.off + h);
+            proj = r > 0 && (!A.row_n || n > 0);
         }
     }
     __device__ long long bh(const FlushArgs &A) const { return (long long)b * A.H + h; }
@@ -154,8 +175,8 @@ template <int KIND>
 __device__ __forceinline__ void issue_item(const FlushArgs &A, const Cursor &it, int nslab, float *Sbuf,
                                            float *T, const FlushCarve &cv, uint64_t *bar, int lane, bool keys)
 {
-    const int V = A.V, VS = A.VS, W = A.W, n = A.n;
-    const bool needed = n > 0 || it.r > 0;
+    const int V = A.V, VS = A.VS, W = A.W, n = it.n;
+    const bool needed = n > 0 || it.proj;
     if (KIND != SKETCHSSM_MAMBA2) keys = true;
     if (lane == 0) {
         uint32_t bytes = 0;
@@ -292,7 +313,7 @@ __global__ void __launch_bounds__(FLUSH_MAXT, 2)
 flush_kernel(const FlushArgs A)
 {
     extern __shared__ __align__(128) unsigned char fsm_raw[];
-    const int V = A.V, W = A.W, n = A.n, VS = A.VS;
+    const int V = A.V, W = A.W, VS = A.VS;
     const int nslab = V / VS;
     const int ncw = VS / 16;  // compute warps
     const FlushCarve cv = flush_carve(KIND, VS, W, A.rcap);
@@ -390,7 +411,7 @@ flush_kernel(const FlushArgs A)
     auto load_scalars = [&](const Cursor &c, float &a, float &bv) {
         a = 1.f;
         bv = 0.f;
-        if (lane < n) {
+        if (lane < c.n) {
             const long long o = c.bh(A) * W + lane;
             if (KIND != SKETCHSSM_KDA) a = __ldg(A.abuf + o);
             if (KIND != SKETCHSSM_MAMBA2) bv = __ldg(A.bbuf + o);
@@ -408,7 +429,7 @@ flush_kernel(const FlushArgs A)
         bool ok = true;         // false once a wait gave up: no more work, barriers only
         for (int j = 0; j < cnt; ++j) {
             const float *T = Tb + (size_t)(j & 1) * cv.tfloats;
-            const int r = cur.r;
+            const int r = cur.r, n = cur.n;
             const bool need_o = new_group(cur);
             ok = ok && staged_wait(full, (uint32_t)(j & 1), A, abort);
             // the state in the accumulator layout: c[mt][nt][2 h + e] = state row
@@ -525,7 +546,7 @@ flush_kernel(const FlushArgs A)
                 ok = ok && staged_wait(obar, o_phase, A, abort);
                 o_phase ^= 1u;
             }
-            if (r > 0 && ok) {
+            if (cur.proj && ok) {
                 float *Yh = A.Y + ((long long)cur.b * A.rtot + cur.off) * V + (long long)cur.slab * VS + col0 + 2 * t;
                 const float *om = Obuf;
                 for (int m0 = 0; m0 < r; m0 += 8) {
@@ -581,7 +602,7 @@ flush_kernel(const FlushArgs A)
     } else {
     for (int j = 0; j < cnt; ++j) {
         const float *T = Tb + (size_t)(j & 1) * cv.tfloats;
-        const int r = cur.r;
+        const int r = cur.r, n = cur.n;
         const bool need_o = new_group(cur);
 
         if (!staged_wait(full, (uint32_t)(j & 1), A, abort)) {
@@ -710,17 +731,17 @@ flush_kernel(const FlushArgs A)
 
         // the sketch rows of this slab: 8 rows at a time, reduced over the 8 row slices
         // by a reduce-scatter that leaves row m0 + ks in lane ks
-        if (r > 0) {
-            if (need_o) {
-                if (!staged_wait(obar, o_phase, A, abort)) {
-                    if (lane == 0) {
-                        *abort = 1;
-                        atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
-                    }
-                    return;
+        if (need_o) {
+            if (!staged_wait(obar, o_phase, A, abort)) {
+                if (lane == 0) {
+                    *abort = 1;
+                    atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
                 }
-                o_phase ^= 1u;
+                return;
             }
+            o_phase ^= 1u;
+        }
+        if (cur.proj) {
             float *Yh = A.Y + ((long long)cur.b * A.rtot + cur.off) * V + (long long)cur.slab * VS +
                         c4 * 4;
             const float *om = Obuf + 4 * ks;

@@ -19,6 +19,7 @@ constexpr int MAX_V = 256;       // value dim
 constexpr int SK_STATUS_DECODE_TIMEOUT = 1;
 constexpr int SK_STATUS_FLUSH_TIMEOUT = 2;
 constexpr int SK_STATUS_STEP_TIMEOUT = 4;
+constexpr int SK_STATUS_BAD_ROW = 8;  // a per-row position or token count out of range
 
 // default bound of a kernel's wait on its own bulk copies (clock cycles, ~1 s)
 constexpr long long DEFAULT_WAIT_CYCLES = 2000000000LL;
@@ -45,6 +46,8 @@ struct DecodeArgs {
     int dots_row;        // Mamba-2 products per (batch row, q/k head): W keys, then cap basis rows
     int maxnh;           // heads per combine item at most
     int coef_cap;        // floats of the combine coefficient stage
+    const int *row_pos;  // per-row buffer positions [B] (device), or null: every row at pos
+    const int *counts;   // layout counts: items of the work list for n at counts[2 + n]
     long long wait_limit;
     int *status;
     const float *q, *k, *v, *a, *beta;
@@ -58,6 +61,7 @@ struct FlushArgs {
     int kind, B, H, Hqk, V, W, G, Rb, cap, n;
     int Hg, hpq;
     int VS;    // column slab of one work item
+    const int *row_n;  // per-row token counts [B] (device), or null: every row applies n
     int rcap;  // the largest sketch rank of the plan (0 if none): basis rows staged per CTA
     const int *rmax;          // [G] largest sketch rank per group
     int *status;              // plan status word (timeouts)

@@ -167,6 +167,8 @@ sk::DecodeArgs decode_args(const sketchssm_plan *p, int pos, const float *q, con
     A.coef_cap = p->geo.coef_cap;
     A.wait_limit = p->wait_limit;
     A.status = p->d_status;
+    A.row_pos = nullptr;
+    A.counts = p->d_counts;
     A.q = q;
     A.k = k;
     A.v = v;
@@ -362,6 +364,9 @@ sketchssm_status sketchssm_plan_check(const sketchssm_plan *p, sketchssm_stream 
     if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream");
     if (flags & sk::SK_STATUS_DECODE_TIMEOUT)
         return fail(SKETCHSSM_ERR_TIMEOUT, "a decode CTA waited past the plan's limit for its bulk copies");
+    if (flags & sk::SK_STATUS_BAD_ROW)
+        return fail(SKETCHSSM_ERR_INVALID_ARG,
+                    "a per-row position or token count was out of range; those rows were left unchanged");
     if (flags & sk::SK_STATUS_STEP_TIMEOUT)
         return fail(SKETCHSSM_ERR_TIMEOUT, "a standard-step CTA waited past the plan's limit for its bulk copies");
     if (flags & sk::SK_STATUS_FLUSH_TIMEOUT)
@@ -395,15 +400,20 @@ sketchssm_status sketchssm_plan_destroy(sketchssm_plan *p)
     return SKETCHSSM_OK;
 }
 
-sketchssm_status sketchssm_flush(const sketchssm_plan *p, float *S, const float *omega, const float *kbuf,
-                                 const float *vbuf, const float *abuf, const float *bbuf, int32_t n_tokens,
-                                 float *Y, sketchssm_stream stream)
+}  // extern "C"
+
+namespace {
+
+sketchssm_status flush_impl(const sketchssm_plan *p, float *S, const float *omega, const float *kbuf,
+                            const float *vbuf, const float *abuf, const float *bbuf, int32_t n_tokens,
+                            const int32_t *row_n, float *Y, sketchssm_stream stream)
 {
     g_last_error.clear();
     sketchssm_status s = check_plan(p);
     if (s != SKETCHSSM_OK) return s;
     const sketchssm_desc &d = p->d;
     if (n_tokens < 0 || n_tokens > d.window) return fail(SKETCHSSM_ERR_INVALID_ARG, "n_tokens outside [0, window]");
+    if (row_n) CHECK_T(row_n, sizeof(int32_t) * (size_t)d.batch, "n_tokens (per row)", false);
     const long long B = d.batch, H = d.heads, Q = d.qk_heads, K = d.key_dim, V = d.value_dim, W = d.window;
     const long long da = d.kind == SKETCHSSM_KDA ? K : 1;
     const bool mamba = d.kind == SKETCHSSM_MAMBA2;
@@ -435,6 +445,7 @@ sketchssm_status sketchssm_flush(const sketchssm_plan *p, float *S, const float 
     A.rmax = p->d_rmax;
     A.status = p->d_status;
     A.wait_limit = p->wait_limit;
+    A.row_n = row_n;
     A.rtot = p->rtot;
     A.rank = p->d_rank;
     A.off = p->d_off;
@@ -447,6 +458,54 @@ sketchssm_status sketchssm_flush(const sketchssm_plan *p, float *S, const float 
     A.Y = Y;
     cudaError_t e = sk::launch_flush(A, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "flush kernel launch");
+    return SKETCHSSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sketchssm_status sketchssm_flush(const sketchssm_plan *p, float *S, const float *omega, const float *kbuf,
+                                 const float *vbuf, const float *abuf, const float *bbuf, int32_t n_tokens,
+                                 float *Y, sketchssm_stream stream)
+{
+    return flush_impl(p, S, omega, kbuf, vbuf, abuf, bbuf, n_tokens, nullptr, Y, stream);
+}
+
+sketchssm_status sketchssm_flush_rows(const sketchssm_plan *p, float *S, const float *omega, const float *kbuf,
+                                      const float *vbuf, const float *abuf, const float *bbuf,
+                                      const int32_t *n_tokens, float *Y, sketchssm_stream stream)
+{
+    g_last_error.clear();
+    if (!n_tokens) return fail(SKETCHSSM_ERR_INVALID_ARG, "n_tokens (per row) is NULL");
+    return flush_impl(p, S, omega, kbuf, vbuf, abuf, bbuf, p ? p->d.window : 0, n_tokens, Y, stream);
+}
+
+sketchssm_status sketchssm_decode_rows(const sketchssm_plan *p, const int32_t *pos, const float *q, const float *k,
+                                       const float *v, const float *a, const float *beta, float *kbuf, float *vbuf,
+                                       float *abuf, float *bbuf, const float *Y, const float *omega, const float *S,
+                                       float *y, sketchssm_stream stream)
+{
+    g_last_error.clear();
+    sketchssm_status s = check_plan(p);
+    if (s != SKETCHSSM_OK) return s;
+    const sketchssm_desc &d = p->d;
+    CHECK_T(pos, sizeof(int32_t) * (size_t)d.batch, "pos (per row)", false);
+    if ((s = check_decode_common(p, 0, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, y)) != SKETCHSSM_OK) return s;
+    const bool any_sketch = p->rtot > 0, any_dense = p->n_dense > 0;
+    CHECK_T(Y, any_sketch ? fbytes(d.batch, p->rtot, d.value_dim) : 0, "Y", !any_sketch);
+    CHECK_T(omega, any_sketch ? fbytes(d.groups, d.basis_rows, d.key_dim) : 0, "omega", !any_sketch);
+    CHECK_T(S, any_dense ? fbytes(d.batch, d.heads, d.key_dim, d.value_dim) : 0, "S", !any_dense);
+    sk::DecodeArgs A = decode_args(p, 0, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, Y, omega, S, y, 0);
+    // every row reads its own work list (the launch covers the longest)
+    A.row_pos = pos;
+    A.work = p->d_work;
+    A.rec = p->d_rec;
+    int most = 0;
+    for (int c : p->h_items) most = c > most ? c : most;
+    A.n_items = most;
+    cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     return SKETCHSSM_OK;
 }
 

@@ -10,7 +10,8 @@ from typing import Optional, Sequence
 import numpy as np
 import torch
 
-from ._binding import Plan, sketchssm_decode, sketchssm_dense_decode, sketchssm_flush, sketchssm_step
+from ._binding import (Plan, sketchssm_decode, sketchssm_decode_rows, sketchssm_dense_decode, sketchssm_flush,
+                       sketchssm_flush_rows, sketchssm_step)
 
 
 def _dev(x, device) -> torch.Tensor:
@@ -61,6 +62,19 @@ class SketchLayer:
         sketchssm_dense_decode(self.plan, pos, q, k, v, a, beta, self.kbuf, self.vbuf, self.abuf,
                                self.bbuf, self.S, y, stream)
         return y
+
+    def decode_rows(self, pos: torch.Tensor, q, k, v, a, beta: Optional[torch.Tensor] = None, out=None,
+                    stream=None) -> torch.Tensor:
+        """Decode with a buffer position per batch row (pos: int32 [B] on the device)."""
+        y = self.y if out is None else out
+        sketchssm_decode_rows(self.plan, pos, q, k, v, a, beta, self.kbuf, self.vbuf, self.abuf, self.bbuf,
+                              self.Y, self.omega, self.S, y, stream)
+        return y
+
+    def flush_rows(self, n_tokens: torch.Tensor, stream=None) -> None:
+        """Flush each batch row's first n_tokens[b] buffered tokens (int32 [B] on the device)."""
+        sketchssm_flush_rows(self.plan, self.S, self.omega, self.kbuf, self.vbuf, self.abuf, self.bbuf,
+                             n_tokens, self.Y, stream)
 
     def standard_step(self, q, k, v, a, beta: Optional[torch.Tensor] = None, out=None,
                       stream=None) -> torch.Tensor:
