@@ -489,9 +489,10 @@ def run_reference(args, cfg) -> None:
 
 def run_profile_case(args, cfg) -> None:
     """A small single-layer run for a profiler (ncu -k <kernel> -s <skip> -c <count>):
-    flush(0), then `--steps` window cycles of W sketch decodes and a flush, with no timing
-    and no JSON line.  Launch order: the initial flush, then per cycle W x (products
-    kernel, combine kernel) and the flush."""
+    flush(0), then `--steps` window cycles of W sketch decodes and a flush, then two
+    standard per-step decodes, with no timing and no JSON line.  Launch order: the
+    initial flush, per cycle W x (products kernel, combine kernel) and the flush, then
+    the two step kernels."""
     import torch
     import rank_state_read_b200 as rs
     rank = synth.layer_rank_table(cfg)
@@ -506,6 +507,9 @@ def run_profile_case(args, cfg) -> None:
             x = xs[p]
             layer.decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
         layer.flush(cfg.W)
+    for p in range(2):  # then two standard per-step decodes (step_kernel)
+        x = xs[p]
+        layer.standard_step(x["q"], x["k"], x["v"], x["a"], x["beta"])
     torch.cuda.synchronize()
     layer.plan.check()
     layer.close()

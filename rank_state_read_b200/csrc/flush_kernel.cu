@@ -229,15 +229,6 @@ __device__ __forceinline__ void issue_item(const FlushArgs &A, const Cursor &it,
     }
 }
 
-// s += c * x, for the 4 rows of a row quad held as s[0..3] and c = (c.x .. c.w)
-__device__ __forceinline__ void quad_rank1(float4 *s, float4 c, float4 x)
-{
-    fma4(s[0], c.x, x);
-    fma4(s[1], c.y, x);
-    fma4(s[2], c.z, x);
-    fma4(s[3], c.w, x);
-}
-
 // acc += sum_e c_e s[e] over a row quad
 __device__ __forceinline__ void quad_dot(float4 &acc, float4 c, const float4 *s)
 {
@@ -600,74 +591,40 @@ flush_kernel(const FlushArgs A)
             atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
         }
     } else {
-    for (int j = 0; j < cnt; ++j) {
-        const float *T = Tb + (size_t)(j & 1) * cv.tfloats;
-        const int r = cur.r, n = cur.n;
-        const bool need_o = new_group(cur);
+        for (int j = 0; j < cnt; ++j) {
+            const float *T = Tb + (size_t)(j & 1) * cv.tfloats;
+            const int r = cur.r, n = cur.n;
+            const bool need_o = new_group(cur);
 
-        if (!staged_wait(full, (uint32_t)(j & 1), A, abort)) {
-            if (lane == 0) {
-                *abort = 1;
-                atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
-            }
-            return;
-        }
-        float4 s[16];
-        {
-            const float *sb = Sbuf + (size_t)ks * (4 * VS + 4) + c4 * 4;
-#pragma unroll
-            for (int q = 0; q < QROWS; ++q)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) s[4 * q + e] = lds4(sb + (size_t)q * 8 * (4 * VS + 4) + e * VS);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty);
-
-        // the next item's scalars, one item ahead
-        Cursor nxt = cur;
-        float a_n = 1.f, b_n = 0.f;
-        if (j + 1 < cnt) {
-            nxt.next(A, nslab);
-            load_scalars(nxt, a_n, b_n);
-        }
-
-        // the update
-        const float *kt = T + cv.tkeys + 4 * ks;
-        const float *vt = T + cv.tv + c4 * 4;
-        if (KIND == SKETCHSSM_MAMBA2) {
-            if (n > 0) {
-                float P = a_l;  // prod of a_i over the lanes (lanes >= n hold 1)
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) P *= __shfl_xor_sync(0xffffffffu, P, o);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    s[q].x *= P; s[q].y *= P; s[q].z *= P; s[q].w *= P;
+            if (!staged_wait(full, (uint32_t)(j & 1), A, abort)) {
+                if (lane == 0) {
+                    *abort = 1;
+                    atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
                 }
-                // newest token first, w_i = prod_{j>i} a_j; token i-1's key and value
-                // are read from shared memory while token i's products issue
-                float w = 1.f;
-                float4 vv = lds4(vt + (n - 1) * VS), kq[QROWS];
-#pragma unroll
-                for (int q = 0; q < QROWS; ++q) kq[q] = lds4(kt + (n - 1) * KDIM + q * 32);
-                for (int i = n - 1; i >= 0; --i) {
-                    float4 vn = vv, kn[QROWS];
-#pragma unroll
-                    for (int q = 0; q < QROWS; ++q) kn[q] = kq[q];
-                    if (i > 0) {
-                        vn = lds4(vt + (i - 1) * VS);
-#pragma unroll
-                        for (int q = 0; q < QROWS; ++q) kn[q] = lds4(kt + (i - 1) * KDIM + q * 32);
-                    }
-                    vv.x *= w; vv.y *= w; vv.z *= w; vv.w *= w;
-#pragma unroll
-                    for (int q = 0; q < QROWS; ++q) quad_rank1(s + 4 * q, kq[q], vv);
-                    w *= __shfl_sync(0xffffffffu, a_l, i);
-                    vv = vn;
-#pragma unroll
-                    for (int q = 0; q < QROWS; ++q) kq[q] = kn[q];
-                }
+                return;
             }
-        } else {
+            float4 s[16];
+            {
+                const float *sb = Sbuf + (size_t)ks * (4 * VS + 4) + c4 * 4;
+#pragma unroll
+                for (int q = 0; q < QROWS; ++q)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) s[4 * q + e] = lds4(sb + (size_t)q * 8 * (4 * VS + 4) + e * VS);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty);
+
+            // the next item's scalars, one item ahead
+            Cursor nxt = cur;
+            float a_n = 1.f, b_n = 0.f;
+            if (j + 1 < cnt) {
+                nxt.next(A, nslab);
+                load_scalars(nxt, a_n, b_n);
+            }
+
+            // the update
+            const float *kt = T + cv.tkeys + 4 * ks;
+            const float *vt = T + cv.tv + c4 * 4;
             const float *at = T + cv.ta + 4 * ks;
             for (int i = 0; i < n; ++i) {
                 const float *ki = kt + i * KDIM;
@@ -719,59 +676,58 @@ flush_kernel(const FlushArgs A)
                     }
                 }
             }
-        }
-        const long long bh = cur.bh(A);
-        if (n > 0) {
-            float *Sg = A.S + (bh * KDIM + 4 * ks) * V + (long long)cur.slab * VS + c4 * 4;
+            const long long bh = cur.bh(A);
+            if (n > 0) {
+                float *Sg = A.S + (bh * KDIM + 4 * ks) * V + (long long)cur.slab * VS + c4 * 4;
 #pragma unroll
-            for (int q = 0; q < QROWS; ++q)
+                for (int q = 0; q < QROWS; ++q)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) st4(Sg + (long long)(32 * q + e) * V, s[4 * q + e]);
-        }
+                    for (int e = 0; e < 4; ++e) st4(Sg + (long long)(32 * q + e) * V, s[4 * q + e]);
+            }
 
-        // the sketch rows of this slab: 8 rows at a time, reduced over the 8 row slices
-        // by a reduce-scatter that leaves row m0 + ks in lane ks
-        if (need_o) {
-            if (!staged_wait(obar, o_phase, A, abort)) {
-                if (lane == 0) {
-                    *abort = 1;
-                    atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
-                }
-                return;
-            }
-            o_phase ^= 1u;
-        }
-        if (cur.proj) {
-            float *Yh = A.Y + ((long long)cur.b * A.rtot + cur.off) * V + (long long)cur.slab * VS +
-                        c4 * 4;
-            const float *om = Obuf + 4 * ks;
-            const bool u2 = ks & 4, u1 = ks & 2, u0 = ks & 1;
-            for (int m0 = 0; m0 < r; m0 += 8) {
-                float4 p[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    float4 x0 = zero4(), x1 = zero4();
-                    if (m0 + u < r) {
-                        const float *o = om + (m0 + u) * KDIM;
-                        quad_dot(x0, lds4(o), s + 0);
-                        quad_dot(x1, lds4(o + 32), s + 4);
-                        quad_dot(x0, lds4(o + 64), s + 8);
-                        quad_dot(x1, lds4(o + 96), s + 12);
+            // the sketch rows of this slab: 8 rows at a time, reduced over the 8 row slices
+            // by a reduce-scatter that leaves row m0 + ks in lane ks
+            if (need_o) {
+                if (!staged_wait(obar, o_phase, A, abort)) {
+                    if (lane == 0) {
+                        *abort = 1;
+                        atomicOr(A.status, SK_STATUS_FLUSH_TIMEOUT);
                     }
-                    p[u] = add4(x0, x1);
+                    return;
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) p[u] = rs_step(p[u], p[u + 4], u2, 4);
-#pragma unroll
-                for (int u = 0; u < 2; ++u) p[u] = rs_step(p[u], p[u + 2], u1, 2);
-                p[0] = rs_step(p[0], p[1], u0, 1);
-                if (m0 + ks < r) st4(Yh + (long long)(m0 + ks) * V, p[0]);
+                o_phase ^= 1u;
             }
+            if (cur.proj) {
+                float *Yh = A.Y + ((long long)cur.b * A.rtot + cur.off) * V + (long long)cur.slab * VS +
+                            c4 * 4;
+                const float *om = Obuf + 4 * ks;
+                const bool u2 = ks & 4, u1 = ks & 2, u0 = ks & 1;
+                for (int m0 = 0; m0 < r; m0 += 8) {
+                    float4 p[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        float4 x0 = zero4(), x1 = zero4();
+                        if (m0 + u < r) {
+                            const float *o = om + (m0 + u) * KDIM;
+                            quad_dot(x0, lds4(o), s + 0);
+                            quad_dot(x1, lds4(o + 32), s + 4);
+                            quad_dot(x0, lds4(o + 64), s + 8);
+                            quad_dot(x1, lds4(o + 96), s + 12);
+                        }
+                        p[u] = add4(x0, x1);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) p[u] = rs_step(p[u], p[u + 4], u2, 4);
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) p[u] = rs_step(p[u], p[u + 2], u1, 2);
+                    p[0] = rs_step(p[0], p[1], u0, 1);
+                    if (m0 + ks < r) st4(Yh + (long long)(m0 + ks) * V, p[0]);
+                }
+            }
+            cur = nxt;
+            a_l = a_n;
+            b_l = b_n;
         }
-        cur = nxt;
-        a_l = a_n;
-        b_l = b_n;
-    }
     }
 }
 
