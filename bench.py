@@ -424,7 +424,10 @@ def run_ours(args, cfg) -> None:
         "speedup_vs_dense_read": round(mean_dd_us / mean_dec_us, 3),
         "traffic_ratio_dense_over_sketch": round(dd_bytes / len(dd) / (dec_bytes / len(dec)), 3),
         "standard_step": {"step_us": round(mean_st_us, 2), "hbm_gbs": round(st_gbs, 1),
-                          "frac": round(st_gbs / peak, 4), "tok_s": round(cfg.B / (mean_st_us * 1e-6), 1)},
+                          "frac": round(st_gbs / peak, 4), "tok_s": round(cfg.B / (mean_st_us * 1e-6), 1),
+                          "algorithmic_bytes_per_launch": step_bytes(cfg),
+                          "traffic": (lambda tr: None if tr is None else tr["dram_bytes_per_launch_full_size"])(
+                              kernel_traffic("sketchssm_step"))},
         "speedup_vs_standard_step": round(cfg.W * mean_st_us / (cfg.W * mean_dec_us + mean_fl_us), 3),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d // ke,
                 "d2h_bytes_per_step": d2h // ke,

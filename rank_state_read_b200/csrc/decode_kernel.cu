@@ -113,12 +113,17 @@ dots_kernel_mamba2(const DecodeArgs A)
     const int rows = A.cm_rows;
     const int q = blockIdx.x, b0 = blockIdx.y * rows;
     const int nb = min(rows, A.B - b0);
-    // buffer position of each of the CTA's rows (-1: a bad per-row position, row skipped)
-    __shared__ int rpos[CM_MAXROWS];
-    if (tid < nb) rpos[tid] = row_position(A, b0 + tid);
-    __syncthreads();
-    int nmax = 0;  // key slots in use in any of the rows (all rows alike: pos + 1)
-    for (int bl = 0; bl < nb; ++bl) nmax = max(nmax, rpos[bl] + 1);
+    // buffer position of each of the CTA's rows (-1: a bad per-row position, row
+    // skipped); all rows at the call's pos unless the call gives per-row positions
+    __shared__ int rpos_s[CM_MAXROWS];
+    int nmax = A.pos + 1;  // key slots in use in any of the rows
+    if (A.row_pos) {
+        if (tid < nb) rpos_s[tid] = row_position(A, b0 + tid);
+        __syncthreads();
+        nmax = 0;
+        for (int bl = 0; bl < nb; ++bl) nmax = max(nmax, rpos_s[bl] + 1);
+    }
+    auto rpos = [&](int bl) { return A.row_pos ? rpos_s[bl] : A.pos; };
     const int g = (q * hpq) / A.Hg;
     const CmCarve cv = cm_carve(cap, W, rows);
     float *om = reinterpret_cast<float *>(cms + cv.om);  // [rq][OPAD]
@@ -136,7 +141,7 @@ dots_kernel_mamba2(const DecodeArgs A)
         cp_async16(qs + bl * OPAD + c * 4, A.q + ((long long)(b0 + bl) * A.Hqk + q) * KDIM + c * 4);
     }
     for (int x = tid; x < nb * nmax * (KDIM / 4); x += CM_THREADS) {
-        const int c = x & 31, r = x >> 5, bl = r / nmax, i = r - bl * nmax, pos = rpos[bl];
+        const int c = x & 31, r = x >> 5, bl = r / nmax, i = r - bl * nmax, pos = rpos(bl);
         if (i > pos) continue;
         const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
         cp_async16(ks + bl * cv.kblock + i * OPAD + c * 4,
@@ -146,8 +151,8 @@ dots_kernel_mamba2(const DecodeArgs A)
     // unused entries of the rows: 0
     for (int x = tid; x < nb * dr; x += CM_THREADS) {
         const int bl = x / dr, e = x - bl * dr;
-        if (rpos[bl] < 0) continue;
-        if ((e > rpos[bl] && e < W) || e >= W + rq) A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + e] = 0.f;
+        if (rpos(bl) < 0) continue;
+        if ((e > rpos(bl) && e < W) || e >= W + rq) A.scratch[((long long)(b0 + bl) * A.Hqk + q) * dr + e] = 0.f;
     }
     cp_async_wait<0>();
     __syncthreads();
@@ -155,7 +160,7 @@ dots_kernel_mamba2(const DecodeArgs A)
     // task (row rr, batch row): rr < nmax a key slot, else basis row rr - nmax
     for (int t = tid; t < (nmax + rq) * nb; t += CM_THREADS) {
         const int rr = t / nb, bl = t - rr * nb;
-        if (rr < nmax && rr > rpos[bl]) continue;
+        if (rr < nmax && rr > rpos(bl)) continue;
         const float *row = rr < nmax ? ks + bl * cv.kblock + rr * OPAD : om + (size_t)(rr - nmax) * OPAD;
         const float *qb = qs + (size_t)bl * OPAD;
         float4 acc = zero4();
@@ -172,7 +177,7 @@ dots_kernel_mamba2(const DecodeArgs A)
     }
     // the step's key goes to buffer slot pos (from the stage)
     for (int x = tid; x < nb * (KDIM / 4); x += CM_THREADS) {
-        const int bl = x >> 5, c = x & 31, pos = rpos[bl];
+        const int bl = x >> 5, c = x & 31, pos = rpos(bl);
         if (pos < 0) continue;
         const long long qrow = (long long)(b0 + bl) * A.Hqk + q;
         st4(A.kbuf + (qrow * W + pos) * KDIM + c * 4, lds4(ks + bl * cv.kblock + pos * OPAD + c * 4));
