@@ -6,11 +6,13 @@ it and shares no code with it.
 
 * ``sketch_oracle.c`` : the algorithm in its steps (flush, sketch, replay, read),
   plain fp64 loops, compiled by ``oracle/build.py``; also the standard per-step
-  recurrent decode (``standard_step``), the baseline the paper compares against.
+  recurrent decode (``standard_step``), the baseline the paper compares against,
+  and the prefill handoff (``prefill``: a prompt's tokens applied to the state in
+  order, after which ``OracleLayer.prefill`` forms the sketch with the n = 0 flush).
 * ``brute``           : the plain definitions on tiny inputs (explicit matrices).
 
 Parity is pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py``;
 nothing here is "parity unpinned" except the accuracy of a rank-r sketch against the
 exact read on real models (that needs a calibrated basis the pages do not publish).
 """
-from .core import OracleLayer, layout, load_library, num_threads, standard_step, trajectory  # noqa: F401
+from .core import OracleLayer, layout, load_library, num_threads, prefill, standard_step, trajectory  # noqa: F401

@@ -40,6 +40,8 @@ def _load():
                                       ctypes.c_int32, P]
         lib.oracle_step.restype = None
         lib.oracle_step.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, P, P, P]
+        lib.oracle_prefill.restype = None
+        lib.oracle_prefill.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int32, P, P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -120,6 +122,12 @@ class OracleLayer:
                              _p(self.S), _p(self.omega), _p(self.kbuf), _p(self.vbuf),
                              _p(self.abuf), _p(self.bbuf), n, _p(self.Y))
 
+    def prefill(self, prompt: dict) -> None:
+        """Prefill handoff: apply the prompt's tokens to S in order (``prefill``), then
+        form Y from the new state (the n = 0 flush).  The buffer is left alone."""
+        prefill(self.kind, self.S, prompt, self.dims.Hqk, lib=self._lib)
+        self.flush(0)
+
     def decode(self, pos: int, inp: dict, dense_all: bool = False) -> np.ndarray:
         """Append the step's token at slot ``pos`` and return y [B][H][V]."""
         assert 0 <= pos < self.dims.W
@@ -151,6 +159,24 @@ def standard_step(kind: str, S: np.ndarray, inp: dict, Hqk: int, lib=None) -> np
     y = np.empty((B, H, V))
     (lib or _load()).oracle_step(ctypes.byref(dims), _p(S), _p(q), _p(k), _p(v), _p(a), _p(beta), _p(y))
     return y
+
+
+def prefill(kind: str, S: np.ndarray, prompt: dict, Hqk: int, lib=None) -> None:
+    """Apply a prompt's tokens to the fp64 state ``S`` [B][H][K][V] in place, in order.
+
+    ``prompt`` is token-major: k [B][T][Hqk][K], v [B][T][H][V], a [B][T][H]
+    (KDA [B][T][H][K]), beta [B][T][H] (None for Mamba-2)."""
+    assert S.dtype == np.float64 and S.flags.c_contiguous
+    B, H, K, V = S.shape
+    k, v, a = (_f64(prompt[x]) for x in ("k", "v", "a"))
+    beta = None if prompt.get("beta") is None else _f64(prompt["beta"])
+    T = k.shape[1]
+    assert k.shape == (B, T, Hqk, K) and v.shape == (B, T, H, V)
+    assert a.shape == ((B, T, H, K) if kind == "kda" else (B, T, H))
+    if kind != "mamba2":
+        assert beta is not None and beta.shape == (B, T, H)
+    dims = _Dims(KIND_ID[kind], B, H, Hqk, K, V, 1, 1, 1)
+    (lib or _load()).oracle_prefill(ctypes.byref(dims), T, _p(S), _p(k), _p(v), _p(a), _p(beta))
 
 
 def trajectory(layer: OracleLayer, inputs: Iterable[dict], *, dense_all: bool = False,

@@ -268,6 +268,52 @@ void oracle_step(const oracle_dims *d, double *S, const double *q, const double 
     }
 }
 
+/* ------------------------------------------------------------------ prefill
+ * Prefill handoff, the step before decoding.  The pages say only that every update
+ * reaches the full state [ABS, write-full]; how a prompt is taken in is left to the
+ * model's own kernels, so the plain reading is used: the prompt's T tokens are applied
+ * to the state one after another, t = 0 .. T-1, with the transition table above,
+ * S <- M_t S + beta_t k_t v_t^T.  The caller then forms the sketch with
+ * oracle_flush(n = 0); the window buffer is not touched and decoding starts at
+ * pos = 0.  Prompt layout (token-major): pk [B][T][Hqk][K], pv [B][T][H][V],
+ * pa [B][T][H] (KDA [B][T][H][K]), pb [B][T][H] (unused for Mamba-2). */
+void oracle_prefill(const oracle_dims *d, int32_t T, double *S, const double *pk, const double *pv,
+                    const double *pa, const double *pb)
+{
+    const int64_t K = d->K, V = d->V, H = d->H;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < d->B; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            const int64_t qh = (h * d->Hqk) / H;
+            double *St = S + (b * H + h) * K * V;
+            double *ev = (double *)malloc(sizeof(double) * V);
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t bth = (b * T + t) * H + h; /* token t of row b, head h */
+                const double *kp = pk + ((b * T + t) * d->Hqk + qh) * K;
+                const double *vp = pv + bth * V;
+                if (d->kind == ORACLE_MAMBA2) {
+                    const double ap = pa[bth];
+                    for (int64_t r = 0; r < K; ++r)
+                        for (int64_t c = 0; c < V; ++c) St[r * V + c] = ap * St[r * V + c] + kp[r] * vp[c];
+                    continue;
+                }
+                const double bp = pb[bth];
+                for (int64_t c = 0; c < V; ++c) { /* (k_t^T S)_c before the update */
+                    double acc = 0.0;
+                    for (int64_t r = 0; r < K; ++r) acc += kp[r] * St[r * V + c];
+                    ev[c] = acc;
+                }
+                for (int64_t r = 0; r < K; ++r) {
+                    const double ap = (d->kind == ORACLE_KDA) ? pa[bth * K + r] : pa[bth];
+                    for (int64_t c = 0; c < V; ++c)
+                        St[r * V + c] = ap * (St[r * V + c] - bp * kp[r] * ev[c]) + bp * kp[r] * vp[c];
+                }
+            }
+            free(ev);
+        }
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -14,10 +14,12 @@ from .gen import (  # noqa: F401
     basis,
     basis_fp64,
     config,
+    device_prompt_inputs,
     device_state,
     device_step_inputs,
     init_state,
     layer_rank_table,
+    prompt_inputs,
     rank_table,
     stack_rank_tables,
     step_inputs,

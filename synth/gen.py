@@ -32,6 +32,7 @@ _TAG_BASIS = 1
 _TAG_INIT = 2
 _TAG_RANKS = 3
 _TAG_STEP = 4
+_TAG_PROMPT = 5
 
 KINDS = ("mamba2", "gdn", "kda")
 
@@ -232,6 +233,36 @@ def step_inputs(cfg: Config, step: int, rows: Iterable[int], layer: int = 0) -> 
     return {"q": q, "k": k, "v": v, "a": a, "beta": beta}
 
 
+def prompt_inputs(cfg: Config, T: int, rows: Iterable[int], layer: int = 0) -> dict:
+    """A prompt of ``T`` tokens for the given batch rows (float32, token-major).
+
+    k: [n][T][Hqk][K], v: [n][T][H][V], a: [n][T][H] (KDA [n][T][H][K]),
+    beta: [n][T][H] (None for Mamba-2); every token drawn with the distributions of
+    ``step_inputs`` (no query: a prompt only writes the state), from its own stream
+    per (row, token).
+    """
+    rows = list(rows)
+    n = len(rows)
+    k = np.empty((n, T, cfg.Hqk, cfg.K), np.float32)
+    v = np.empty((n, T, cfg.H, cfg.V), np.float32)
+    a = np.empty((n, T, cfg.H, cfg.K) if cfg.kda else (n, T, cfg.H), np.float32)
+    beta = np.empty((n, T, cfg.H), np.float32) if cfg.has_beta else None
+    lo = np.nextafter(np.float32(0.9), np.float32(1.0))
+    hi = np.nextafter(np.float32(1.0), np.float32(0.0))
+    for j, b in enumerate(rows):
+        for t in range(T):
+            rng = np.random.default_rng([cfg.seed, _TAG_PROMPT, layer, t, b])
+            k[j, t] = _unit_rows(rng.standard_normal((cfg.Hqk, cfg.K)))
+            v[j, t] = rng.standard_normal((cfg.H, cfg.V))
+            if cfg.kda:
+                a[j, t] = np.clip((0.9 + 0.1 * rng.uniform(size=(cfg.H, cfg.K))).astype(np.float32), lo, hi)
+            else:
+                a[j, t] = np.exp(-_softplus(rng.standard_normal(cfg.H)) * 0.05)
+            if beta is not None:
+                beta[j, t] = 1.0 / (1.0 + np.exp(-rng.standard_normal(cfg.H)))
+    return {"k": k, "v": v, "a": a, "beta": beta}
+
+
 # ----------------------------------------------------------------------------- device draws
 
 def device_state(cfg: Config, seed: int, device) -> "torch.Tensor":
@@ -244,6 +275,27 @@ def device_state(cfg: Config, seed: int, device) -> "torch.Tensor":
     S = torch.empty((cfg.B, cfg.H, cfg.K, cfg.V), dtype=torch.float32, device=device)
     S.normal_(0.0, 0.1, generator=g)
     return S
+
+
+def device_prompt_inputs(cfg: Config, T: int, seed: int, device) -> dict:
+    """A prompt of ``T`` tokens with the distributions of ``prompt_inputs``, drawn on
+    ``device`` (token-major, as ``prompt_inputs``)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    f32 = dict(dtype=torch.float32, device=device)
+    z = torch.randn((cfg.B, T, cfg.Hqk, cfg.K), generator=g, **f32)
+    out = {"k": z / z.norm(dim=-1, keepdim=True),
+           "v": torch.randn((cfg.B, T, cfg.H, cfg.V), generator=g, **f32)}
+    if cfg.kda:
+        lo = float(np.nextafter(np.float32(0.9), np.float32(1.0)))
+        hi = float(np.nextafter(np.float32(1.0), np.float32(0.0)))
+        out["a"] = (0.9 + 0.1 * torch.rand((cfg.B, T, cfg.H, cfg.K), generator=g, **f32)).clamp_(lo, hi)
+    else:
+        out["a"] = torch.exp(-torch.nn.functional.softplus(torch.randn((cfg.B, T, cfg.H), generator=g, **f32)) * 0.05)
+    out["beta"] = (torch.sigmoid(torch.randn((cfg.B, T, cfg.H), generator=g, **f32))
+                   if cfg.has_beta else None)
+    return out
 
 
 def device_step_inputs(cfg: Config, seed: int, device) -> dict:

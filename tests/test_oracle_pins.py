@@ -392,3 +392,150 @@ def test_step_mutations_are_caught(name, old, new, kind, tmp_path):
     obuild.build(force=True, src=str(mutated), out=out)
     lib = oracle.load_library(out)
     assert check_step_against_brute(tiny_cfg(kind, Hqk=2 if kind == "mamba2" else None), T=7, lib=lib) > 1e-6
+
+
+# --------------------------------------------------------------------------- prefill handoff
+
+def head_keys(cfg, k):
+    """Token-major keys [B][T][Hqk][K] seen per state head: [B][T][H][K]."""
+    return np.asarray(k, np.float64)[:, :, (np.arange(cfg.H) * cfg.Hqk) // cfg.H, :]
+
+
+def prefilled(cfg, T, prompt=None, lib=None):
+    rows = list(range(cfg.B))
+    S = np.ascontiguousarray(synth.init_state(cfg, rows), dtype=np.float64)
+    S0 = S.copy()
+    prompt = synth.prompt_inputs(cfg, T, rows) if prompt is None else prompt
+    oracle.prefill(cfg.kind, S, prompt, cfg.Hqk, lib=lib)
+    return S0, S, prompt
+
+
+def test_prefill_mamba2_closed_form():
+    """Mamba-2 unrolls to S_T = (prod_t a_t) S_0 + sum_t (prod_{j>t} a_j) k_t v_t^T."""
+    cfg = tiny_cfg("mamba2", Hqk=2)
+    T = 2 * cfg.W + 3
+    S0, S, p = prefilled(cfg, T)
+    a = p["a"].astype(np.float64)
+    w = np.ones_like(a)  # w[:, t] = prod_{j > t} a_j
+    for t in range(T - 2, -1, -1):
+        w[:, t] = w[:, t + 1] * a[:, t + 1]
+    P = w[:, 0] * a[:, 0]
+    exp = P[:, :, None, None] * S0 + np.einsum("bth,bthk,bthv->bhkv", w, head_keys(cfg, p["k"]),
+                                               p["v"].astype(np.float64))
+    assert rel(S, exp) < 1e-13
+
+
+@pytest.mark.parametrize("kind", ["gdn", "kda"])
+def test_prefill_delta_rule_orthonormal_keys(kind):
+    """No decay, beta = 1 and orthonormal keys: each token replaces the state's component
+    along its key, so S_T = (I - sum_t k_t k_t^T) S_0 + sum_t k_t v_t^T."""
+    cfg = tiny_cfg(kind, K=8, Hqk=2)
+    T = 5
+    p = synth.prompt_inputs(cfg, T, range(cfg.B))
+    rng = np.random.default_rng(5)
+    k = np.empty(p["k"].shape)
+    for b in range(cfg.B):
+        for qh in range(cfg.Hqk):
+            Q, _ = np.linalg.qr(rng.standard_normal((cfg.K, cfg.K)))
+            k[b, :, qh, :] = Q[:, :T].T
+    p = dict(p, k=k, a=np.ones(p["a"].shape), beta=np.ones(p["beta"].shape))
+    S0, S, _ = prefilled(cfg, T, prompt=p)
+    kh = head_keys(cfg, k)
+    proj = np.eye(cfg.K) - np.einsum("bthk,bthl->bhkl", kh, kh)
+    exp = np.einsum("bhkl,bhlv->bhkv", proj, S0) + np.einsum("bthk,bthv->bhkv", kh, p["v"].astype(np.float64))
+    assert rel(S, exp) < 1e-12
+
+
+@pytest.mark.parametrize("kind", ["gdn", "kda"])
+def test_prefill_delta_rule_without_writes(kind):
+    """beta = 0 leaves the decays alone: S_T = (prod_t a_t) S_0, per head (GDN) or per
+    key row (KDA)."""
+    cfg = tiny_cfg(kind)
+    T = 7
+    p = synth.prompt_inputs(cfg, T, range(cfg.B))
+    p = dict(p, beta=np.zeros(p["beta"].shape))
+    S0, S, _ = prefilled(cfg, T, prompt=p)
+    P = np.prod(p["a"].astype(np.float64), axis=1)
+    exp = (P[:, :, None, None] if kind == "gdn" else P[:, :, :, None]) * S0
+    assert rel(S, exp) < 1e-13
+
+
+def check_handoff_against_brute(cfg, rank, T, lib=None):
+    """The handoff (prefill, then the n = 0 flush) against the explicit-matrix
+    definition fed the same tokens one step at a time: brute.run_row's state and sketch
+    at its last flush (T a multiple of W)."""
+    rows = list(range(cfg.B))
+    omega = synth.basis_fp64(cfg)
+    S0 = synth.init_state(cfg, rows)
+    p = synth.prompt_inputs(cfg, T, rows)
+    layer = oracle.OracleLayer(cfg.kind, H=cfg.H, Hqk=cfg.Hqk, K=cfg.K, V=cfg.V, W=cfg.W, G=cfg.G,
+                               rank=rank, omega=omega, S0=S0, lib=lib)
+    layer.prefill(p)
+    steps = [{"q": p["k"][:, t], "k": p["k"][:, t], "v": p["v"][:, t], "a": p["a"][:, t],
+              "beta": None if p["beta"] is None else p["beta"][:, t]} for t in range(T)]
+    worst = 0.0
+    for b in rows:
+        bf = brute.run_row(cfg.kind, S0[b], [{x: (None if s[x] is None else s[x][b]) for x in s} for s in steps],
+                           rank, omega, cfg.G, cfg.Hqk, cfg.W)
+        worst = max(worst, rel(layer.S[b], bf["S_flush"][-1]))
+        for h in range(cfg.H):
+            if rank[h] != DENSE:
+                o = layer.off[h]
+                worst = max(worst, rel(layer.Y[b, o:o + rank[h]], bf["Y_flush"][-1][h]))
+    return worst
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+def test_prefill_handoff_brute_force(kind):
+    """State and sketch after a prompt of two windows equal the token-by-token
+    definition with explicit transition matrices."""
+    cfg = tiny_cfg(kind, Hqk=2 if kind == "mamba2" else None)
+    rank = np.array([1, DENSE, 2, 3], np.int32)
+    assert check_handoff_against_brute(cfg, rank, T=2 * cfg.W) < 1e-12
+
+
+def test_prefill_of_no_tokens_is_the_initial_flush():
+    """T = 0: the state is unchanged and Y = Omega_r S_0 for every sketch head."""
+    cfg = tiny_cfg("gdn")
+    rank = np.array([1, DENSE, 2, 3], np.int32)
+    omega = synth.basis_fp64(cfg)
+    S0 = synth.init_state(cfg, range(cfg.B))
+    layer = oracle.OracleLayer("gdn", H=cfg.H, Hqk=cfg.Hqk, K=cfg.K, V=cfg.V, W=cfg.W, G=cfg.G,
+                               rank=rank, omega=omega, S0=S0)
+    layer.prefill(synth.prompt_inputs(cfg, 0, range(cfg.B)))
+    assert np.array_equal(layer.S, S0.astype(np.float64))
+    for h in range(cfg.H):
+        if rank[h] != DENSE:
+            g = h * cfg.G // cfg.H
+            exp = np.einsum("mk,bkv->bmv", omega[g, :rank[h]], S0[:, h].astype(np.float64))
+            assert rel(layer.Y[:, layer.off[h]:layer.off[h] + rank[h]], exp) < 1e-13
+
+
+PREFILL_MUTATIONS = [
+    ("prefill drops the decay",
+     "St[r * V + c] = ap * St[r * V + c] + kp[r] * vp[c];",
+     "St[r * V + c] = St[r * V + c] + kp[r] * vp[c];", "mamba2"),
+    ("prefill erase sign",
+     "ap * (St[r * V + c] - bp * kp[r] * ev[c])",
+     "ap * (St[r * V + c] + bp * kp[r] * ev[c])", "gdn"),
+    ("prefill tokens in reverse",
+     "const int64_t bth = (b * T + t) * H + h;",
+     "const int64_t bth = (b * T + (T - 1 - t)) * H + h;", "kda"),
+    ("prefill key of the wrong q/k head",
+     "const int64_t qh = (h * d->Hqk) / H;",
+     "const int64_t qh = h % d->Hqk;", "mamba2"),
+]
+
+
+@pytest.mark.parametrize("name,old,new,kind", PREFILL_MUTATIONS, ids=[m[0] for m in PREFILL_MUTATIONS])
+def test_prefill_mutations_are_caught(name, old, new, kind, tmp_path):
+    src = open(obuild.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique: {old!r}"
+    mutated = tmp_path / "mut.c"
+    mutated.write_text(src.replace(old, new))
+    out = str(tmp_path / "libmut.so")
+    obuild.build(force=True, src=str(mutated), out=out)
+    lib = oracle.load_library(out)
+    cfg = tiny_cfg(kind, Hqk=2 if kind == "mamba2" else None)
+    rank = np.array([1, DENSE, 2, 3], np.int32)
+    assert check_handoff_against_brute(cfg, rank, T=2 * cfg.W, lib=lib) > 1e-6
