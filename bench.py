@@ -12,7 +12,9 @@ finds its layer's data in the 126 MB L2 from the previous step.
 Printed JSON line (rank 0): value = tokens per second per SSM layer over all ranks,
 device time (CUDA events, max over ranks), plus the per-kernel roofline of the
 dominant kernel, the dense-read decode baseline, an end-to-end number through the
-C ABI with host-resident inputs, and the fp64 CPU oracle timed on the host cores.
+C ABI with host-resident inputs, the fp64 CPU oracle timed on the host cores, and
+the prefill handoff (a 64-token prompt applied to the state, then its sketch) with the
+prefill kernel's rate against the FP32 pipe's peak.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -82,6 +84,21 @@ def step_bytes(cfg) -> int:
     per_row = (2 * cfg.H * cfg.K * cfg.V + 2 * cfg.Hqk * cfg.K + 2 * cfg.H * cfg.V + cfg.H * da
                + (cfg.H if cfg.has_beta else 0))
     return 4 * cfg.B * per_row
+
+
+PREFILL_T = 64        # prompt tokens of the timed prefill handoff
+FP32_LANES_PER_SM = 128
+SMS = 148
+
+
+def prefill_instr(cfg, T: int) -> int:
+    """Algorithmic FP32 lane instructions of one prefill launch (T tokens into every
+    state element): Mamba-2 2 per element and token (k_i v_j, then a S + that as one
+    FMA); GDN 3 (the k^T S accumulation, beta k times the corrected value, a S + that);
+    KDA 4 (its decay differs per key row, so the correction v - a (k^T S) is formed per
+    element too)."""
+    per = {"mamba2": 2, "gdn": 3, "kda": 4}[cfg.kind]
+    return per * cfg.B * cfg.H * cfg.K * cfg.V * T
 
 
 def flush_bytes(cfg, rank, n: int) -> int:
@@ -338,6 +355,29 @@ def run_ours(args, cfg) -> None:
     barrier()
     st = [a.elapsed_time(b) for a, b in st_ev]
 
+    # ---- prefill handoff on replica 0: a prompt of PREFILL_T tokens applied to the state,
+    # then the sketch formed (sketchssm_prefill); the kernel alone = the call with the
+    # prompt minus the call with none (which only forms the sketch)
+    prompt = synth.device_prompt_inputs(cfg, PREFILL_T, replica_seed(rank_id, 99), dev)
+    pf_ev = {PREFILL_T: [], 0: []}
+    barrier()
+    for it in range(4):
+        for T in (PREFILL_T, 0):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            if T:
+                layers[0].prefill(prompt["k"], prompt["v"], prompt["a"], prompt["beta"])
+            else:
+                rs.sketchssm_prefill(layers[0].plan, 0, None, None, None, None, layers[0].S, layers[0].omega,
+                                     layers[0].Y)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record(stream)
+            if it:  # the first round warms up
+                pf_ev[T].append((e0, e1))
+    barrier()
+    pf_us = {T: 1e3 * sum(a.elapsed_time(b) for a, b in ev) / len(ev) for T, ev in pf_ev.items()}
+    del prompt
+
     # ---- end to end through the C ABI: inputs from pinned host memory, y back to host
     host_in = [{k: (None if v is None else v.cpu().pin_memory()) for k, v in inputs[0][p].items()}
                for p in range(cfg.W)]
@@ -429,6 +469,7 @@ def run_ours(args, cfg) -> None:
                           "traffic": (lambda tr: None if tr is None else tr["dram_bytes_per_launch_full_size"])(
                               kernel_traffic("sketchssm_step"))},
         "speedup_vs_standard_step": round(cfg.W * mean_st_us / (cfg.W * mean_dec_us + mean_fl_us), 3),
+        "prefill": prefill_report(cfg, pf_us, clocks),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d // ke,
                 "d2h_bytes_per_step": d2h // ke,
                 "note": "pinned host inputs copied in and y copied out around every decode call"},
@@ -446,6 +487,22 @@ def run_ours(args, cfg) -> None:
 
 
 # ----------------------------------------------------------------------------- reference arm
+
+def prefill_report(cfg, pf_us: dict, clocks: dict) -> dict:
+    """The prefill handoff's line: its time, prompt tok/s, and the prefill kernel's rate
+    of FP32 lane instructions against the FP32 pipe's peak (148 SMs x 128 lanes x the SM
+    clock seen under load)."""
+    T = PREFILL_T
+    k_us = max(pf_us[T] - pf_us[0], 1e-3)
+    mhz = clocks.get("sm_max_mhz") or 1965.0
+    peak = SMS * FP32_LANES_PER_SM * mhz * 1e6 / 1e12
+    ach = prefill_instr(cfg, T) / (k_us * 1e-6) / 1e12
+    return {"prompt_tokens": T, "handoff_us": round(pf_us[T], 2), "sketch_only_us": round(pf_us[0], 2),
+            "kernel_us": round(k_us, 2), "prompt_tok_s": round(cfg.B * T / (pf_us[T] * 1e-6), 1),
+            "roofline": {"kernel": "sketchssm_prefill", "bound": "alu", "achieved": round(ach, 2),
+                         "peak": round(peak, 2), "unit": "T FP32 lane-instr/s", "frac": round(ach / peak, 4),
+                         "algorithmic_instr_per_launch": prefill_instr(cfg, T)}}
+
 
 def run_reference(args, cfg) -> None:
     """The reference arm of this pipeline is the fp64 CPU oracle as it stands: each
@@ -493,9 +550,9 @@ def run_reference(args, cfg) -> None:
 def run_profile_case(args, cfg) -> None:
     """A small single-layer run for a profiler (ncu -k <kernel> -s <skip> -c <count>):
     flush(0), then `--steps` window cycles of W sketch decodes and a flush, then two
-    standard per-step decodes, with no timing and no JSON line.  Launch order: the
-    initial flush, per cycle W x (products kernel, combine kernel) and the flush, then
-    the two step kernels."""
+    standard per-step decodes and a prefill handoff of 32 tokens, with no timing and no
+    JSON line.  Launch order: the initial flush, per cycle W x (products kernel, combine
+    kernel) and the flush, the two step kernels, then the prefill kernel and its flush."""
     import torch
     import rank_state_read_b200 as rs
     rank = synth.layer_rank_table(cfg)
@@ -513,6 +570,8 @@ def run_profile_case(args, cfg) -> None:
     for p in range(2):  # then two standard per-step decodes (step_kernel)
         x = xs[p]
         layer.standard_step(x["q"], x["k"], x["v"], x["a"], x["beta"])
+    pr = synth.device_prompt_inputs(cfg, 32, 7, "cuda")  # then a prefill handoff of 32 tokens
+    layer.prefill(pr["k"], pr["v"], pr["a"], pr["beta"])
     torch.cuda.synchronize()
     layer.plan.check()
     layer.close()

@@ -280,6 +280,25 @@ sketchssm_status sketchssm_step(const sketchssm_plan *plan, const float *q, cons
                                 const float *v, const float *a, const float *beta, float *S,
                                 float *y, sketchssm_stream stream);
 
+/*
+ * Prefill handoff: the step before decoding.  For every (b, h) the prompt's T tokens
+ * are applied to S in place, in order t = 0 .. T-1, with the decode path's recurrence
+ * S <- M_t S + beta_t k_t v_t^T (paper abstract: every state update reaches the full
+ * state; the pages leave the prompt to the model, so the tokens are applied one after
+ * another).  Then Y is formed from the new state exactly as
+ * sketchssm_flush(n_tokens = 0) forms it.  The window buffer is not read or written:
+ * decoding continues at pos = 0.  T = 0 only forms Y.
+ *  - Prompt layouts (token-major, as a model produces them; 16-byte aligned):
+ *    k [B][T][Hqk][K], v [B][T][H][V], a [B][T][H] (KDA [B][T][H][K]),
+ *    beta [B][T][H] (NULL for Mamba-2).  k, v, a may be NULL when T = 0.
+ *  - S [B][H][K][V] is read and written once whatever T; omega and Y as for
+ *    sketchssm_flush.
+ *  - T < 0 returns SKETCHSSM_ERR_INVALID_ARG; nothing is launched on an error.
+ */
+sketchssm_status sketchssm_prefill(const sketchssm_plan *plan, int32_t T, const float *k, const float *v,
+                                   const float *a, const float *beta, float *S, const float *omega,
+                                   float *Y, sketchssm_stream stream);
+
 /* Static text of a status code. */
 const char *sketchssm_status_string(sketchssm_status status);
 

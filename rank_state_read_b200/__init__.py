@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     sketchssm_flush_rows,
     sketchssm_plan_create,
     sketchssm_plan_destroy,
+    sketchssm_prefill,
     sketchssm_step,
 )
 from .layer import SketchLayer  # noqa: F401

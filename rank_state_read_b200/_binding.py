@@ -24,7 +24,7 @@ STATUS = {0: "SKETCHSSM_OK", 1: "SKETCHSSM_ERR_INVALID_ARG", 2: "SKETCHSSM_ERR_A
 EXPORTS = ("sketchssm_plan_create", "sketchssm_plan_query", "sketchssm_plan_check",
            "sketchssm_plan_set_wait_limit", "sketchssm_plan_destroy", "sketchssm_flush", "sketchssm_decode", "sketchssm_dense_decode",
            "sketchssm_decode_static_scratch", "sketchssm_step", "sketchssm_decode_rows",
-           "sketchssm_flush_rows", "sketchssm_status_string", "sketchssm_last_error")
+           "sketchssm_flush_rows", "sketchssm_prefill", "sketchssm_status_string", "sketchssm_last_error")
 
 
 class SketchSSMError(RuntimeError):
@@ -64,7 +64,8 @@ def load():
     lib.sketchssm_step.argtypes = [P, P, P, P, P, P, P, P, P]
     lib.sketchssm_decode_rows.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
     lib.sketchssm_flush_rows.argtypes = [P, P, P, P, P, P, P, P, P, P]
-    for f in EXPORTS[:12]:
+    lib.sketchssm_prefill.argtypes = [P, I32, P, P, P, P, P, P, P, P]
+    for f in EXPORTS[:13]:
         getattr(lib, f).restype = ctypes.c_int
     lib.sketchssm_status_string.argtypes = [ctypes.c_int]
     lib.sketchssm_status_string.restype = ctypes.c_char_p
@@ -234,6 +235,23 @@ def sketchssm_step(plan: Plan, q, k, v, a, beta, S, y, stream=None) -> None:
         plan.handle, _ptr(q, "q", n("q")), _ptr(k, "k", n("k")), _ptr(v, "v", n("v")), _ptr(a, "a", n("a")),
         _ptr(beta, "beta", n("beta")), _ptr(S, "S", n("S")), _ptr(y, "y", n("y")), _stream(stream)),
         "sketchssm_step")
+
+
+def sketchssm_prefill(plan: Plan, T: int, k, v, a, beta, S, omega, Y, stream=None) -> None:
+    """Prefill handoff (sketchssm_prefill): the prompt's T tokens applied to S in place,
+    then Y formed from the new state.  k [B][T][Hqk][K], v [B][T][H][V], a [B][T][H]
+    (KDA [B][T][H][K]), beta [B][T][H] (None for Mamba-2)."""
+    d, n = plan.desc, plan.numel
+    T = int(T)
+    per_tok = {"k": d.batch * d.qk_heads * d.key_dim, "v": d.batch * d.heads * d.value_dim,
+               "a": n("a"), "beta": d.batch * d.heads}
+    if T == 0:
+        k = v = a = beta = None
+    _check(load().sketchssm_prefill(
+        plan.handle, T, _ptr(k, "k", T * per_tok["k"]), _ptr(v, "v", T * per_tok["v"]),
+        _ptr(a, "a", T * per_tok["a"]), _ptr(beta, "beta", T * per_tok["beta"]),
+        _ptr(S, "S", n("S")), _ptr(omega, "omega", n("omega")), _ptr(Y, "Y", n("Y")), _stream(stream)),
+        "sketchssm_prefill")
 
 
 def _rows(t, name: str, B: int):

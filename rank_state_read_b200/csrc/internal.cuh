@@ -97,6 +97,17 @@ struct StepArgs {
 int step_slab(int V);
 cudaError_t launch_step(const StepArgs &a, cudaStream_t stream);
 
+// Prefill: a prompt of T tokens (token-major k [B][T][Hqk][K], v [B][T][H][V],
+// a [B][T][H] or KDA [B][T][H][K], beta [B][T][H]) applied to S in place; the column
+// slab VS follows step_slab.
+struct PrefillArgs {
+    int kind, B, H, Hqk, V, hpq, T;
+    int VS;
+    const float *k, *v, *a, *beta;
+    float *S;
+};
+cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream);
+
 int flush_slab(int V);
 size_t flush_smem_bytes(int kind, int V, int W, int rcap);
 cudaError_t launch_flush(const FlushArgs &a, cudaStream_t stream);

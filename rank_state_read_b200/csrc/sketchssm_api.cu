@@ -631,6 +631,48 @@ extern "C" sketchssm_status sketchssm_decode_static_scratch(const sketchssm_plan
     return SKETCHSSM_OK;
 }
 
+extern "C" sketchssm_status sketchssm_prefill(const sketchssm_plan *p, int32_t T, const float *k, const float *v,
+                                              const float *a, const float *beta, float *S, const float *omega,
+                                              float *Y, sketchssm_stream stream)
+{
+    g_last_error.clear();
+    sketchssm_status s = check_plan(p);
+    if (s != SKETCHSSM_OK) return s;
+    if (T < 0) return fail(SKETCHSSM_ERR_INVALID_ARG, "T < 0");
+    const sketchssm_desc &d = p->d;
+    const long long B = d.batch, H = d.heads, Q = d.qk_heads, K = d.key_dim, V = d.value_dim;
+    const long long da = d.kind == SKETCHSSM_KDA ? K : 1;
+    const bool mamba = d.kind == SKETCHSSM_MAMBA2;
+    const bool toks = T > 0;
+    if ((long long)B * H * (V / sk::step_slab(d.value_dim)) > 0x7fffffffLL)
+        return fail(SKETCHSSM_ERR_UNSUPPORTED, "batch * heads too large for one prefill launch");
+    CHECK_T(k, toks ? fbytes(B, T, Q, K) : 0, "k", !toks);
+    CHECK_T(v, toks ? fbytes(B, T, H, V) : 0, "v", !toks);
+    CHECK_T(a, toks ? fbytes(B, T, H, da) : 0, "a", !toks);
+    CHECK_T(beta, (toks && !mamba) ? fbytes(B, T, H) : 0, "beta", !toks || mamba);
+    CHECK_T(S, fbytes(B, H, K, V), "S", false);
+    if (toks) {
+        sk::PrefillArgs A;
+        A.kind = d.kind;
+        A.B = d.batch;
+        A.H = d.heads;
+        A.Hqk = d.qk_heads;
+        A.V = d.value_dim;
+        A.hpq = p->hpq;
+        A.T = T;
+        A.VS = sk::step_slab(d.value_dim);
+        A.k = k;
+        A.v = v;
+        A.a = a;
+        A.beta = beta;
+        A.S = S;
+        cudaError_t e = sk::launch_prefill(A, (cudaStream_t)stream);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+    }
+    // the handoff: the sketch of the new state (no buffered tokens)
+    return flush_impl(p, S, omega, nullptr, nullptr, nullptr, nullptr, 0, nullptr, Y, stream);
+}
+
 extern "C" sketchssm_status sketchssm_step(const sketchssm_plan *p, const float *q, const float *k,
                                            const float *v, const float *a, const float *beta, float *S,
                                            float *y, sketchssm_stream stream)

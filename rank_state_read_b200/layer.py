@@ -11,7 +11,7 @@ import numpy as np
 import torch
 
 from ._binding import (Plan, sketchssm_decode, sketchssm_decode_rows, sketchssm_dense_decode, sketchssm_flush,
-                       sketchssm_flush_rows, sketchssm_step)
+                       sketchssm_flush_rows, sketchssm_prefill, sketchssm_step)
 
 
 def _dev(x, device) -> torch.Tensor:
@@ -82,6 +82,12 @@ class SketchLayer:
         y = self.y if out is None else out
         sketchssm_step(self.plan, q, k, v, a, beta, self.S, y, stream)
         return y
+
+    def prefill(self, k, v, a, beta: Optional[torch.Tensor] = None, stream=None) -> None:
+        """Prefill handoff: the prompt (token-major k [B][T][Hqk][K], v [B][T][H][V],
+        a [B][T][H] or KDA [B][T][H][K], beta [B][T][H]) applied to S, then Y formed
+        from the new state; decoding continues at pos = 0."""
+        sketchssm_prefill(self.plan, int(k.shape[1]), k, v, a, beta, self.S, self.omega, self.Y, stream)
 
     def close(self) -> None:
         self.plan.close()

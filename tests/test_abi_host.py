@@ -89,6 +89,7 @@ def test_calls_without_a_plan(lib):
     assert lib.sketchssm_plan_set_wait_limit(None, 1000) == 1
     assert lib.sketchssm_decode_rows(None, *([None] * 14), None) == 1
     assert lib.sketchssm_flush_rows(None, *([None] * 8), None) == 1
+    assert lib.sketchssm_prefill(None, 0, *([None] * 7), None) == 1
     assert lib.sketchssm_plan_check(None, None) == 1
     assert lib.sketchssm_plan_destroy(None) == 0
 
