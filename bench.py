@@ -92,12 +92,14 @@ SMS = 148
 
 
 def prefill_instr(cfg, T: int) -> int:
-    """Algorithmic FP32 lane instructions of one prefill launch (T tokens into every
-    state element): Mamba-2 2 per element and token (k_i v_j, then a S + that as one
-    FMA); GDN 3 (the k^T S accumulation, beta k times the corrected value, a S + that);
-    KDA 4 (its decay differs per key row, so the correction v - a (k^T S) is formed per
-    element too)."""
-    per = {"mamba2": 2, "gdn": 3, "kda": 4}[cfg.kind]
+    """Algorithmic FP32 lane instructions of one prefill launch: the fewest FMA-pipe
+    instructions per state element and prompt token of the forms of the recurrence
+    written out here.  Mamba-2 1: over a chunk S <- P S + sum_i (w_i k_i) v_i^T, one
+    FMA per element and token (the per-chunk scale and key scaling are extra).  GDN 2:
+    with the decay carried as a running scale, k^T S is one FMA and the rank-one write
+    another.  KDA 3: its decay differs per key row, so the write takes two FMAs (the
+    erase term and the new value) besides the k^T S one."""
+    per = {"mamba2": 1, "gdn": 2, "kda": 3}[cfg.kind]
     return per * cfg.B * cfg.H * cfg.K * cfg.V * T
 
 

@@ -118,26 +118,37 @@ __global__ void __launch_bounds__(PF_MAXT) prefill_kernel(const PrefillArgs A)
         const float *ac = as_ + st * PF_CHUNK * da;
         const float *bc = bs_ + st * PF_CHUNK;
         const int n = min(PF_CHUNK, T - c * PF_CHUNK);
-        for (int i = 0; i < n; ++i) {
-            float4 kq[4];
+        if (KIND == SKETCHSSM_MAMBA2) {
+            // the chunk at once: S <- P S + sum_i w_i k_i v_i^T with w_i = prod_{j>i} a_j
+            // and P = prod_j a_j over the chunk's tokens, so that a token costs one FMA
+            // per state element (its key is scaled by w_i first)
+            float P = 1.f;
+            for (int i = 0; i < n; ++i) P *= ac[i];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) kq[q] = lds4(kc + i * KDIM + 4 * ks + 32 * q);
-            const float4 vv = lds4(vc + i * VS + c4 * 4);
-            if (KIND == SKETCHSSM_MAMBA2) {
-                const float at = ac[i];
+            for (int x = 0; x < 16; ++x) {
+                s[x].x *= P;
+                s[x].y *= P;
+                s[x].z *= P;
+                s[x].w *= P;
+            }
+            float w = 1.f;  // w_i, walking the chunk newest first
+            for (int i = n - 1; i >= 0; --i) {
+                const float4 vv = lds4(vc + i * VS + c4 * 4);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float kk[4] = {kq[q].x, kq[q].y, kq[q].z, kq[q].w};
+                    const float4 k4 = lds4(kc + i * KDIM + 4 * ks + 32 * q);
+                    const float kk[4] = {w * k4.x, w * k4.y, w * k4.z, w * k4.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float4 &t = s[4 * q + e];
-                        t.x = fmaf(at, t.x, kk[e] * vv.x);
-                        t.y = fmaf(at, t.y, kk[e] * vv.y);
-                        t.z = fmaf(at, t.z, kk[e] * vv.z);
-                        t.w = fmaf(at, t.w, kk[e] * vv.w);
-                    }
+                    for (int e = 0; e < 4; ++e) fma4(s[4 * q + e], kk[e], vv);
                 }
-            } else {
+                w *= ac[i];
+            }
+        } else {
+            for (int i = 0; i < n; ++i) {
+                float4 kq[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) kq[q] = lds4(kc + i * KDIM + 4 * ks + 32 * q);
+                const float4 vv = lds4(vc + i * VS + c4 * 4);
                 // d = S^T k for this column chunk, before the update
                 float4 d = zero4();
 #pragma unroll
