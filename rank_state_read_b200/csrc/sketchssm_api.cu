@@ -651,6 +651,10 @@ extern "C" sketchssm_status sketchssm_prefill(const sketchssm_plan *p, int32_t T
     CHECK_T(a, toks ? fbytes(B, T, H, da) : 0, "a", !toks);
     CHECK_T(beta, (toks && !mamba) ? fbytes(B, T, H) : 0, "beta", !toks || mamba);
     CHECK_T(S, fbytes(B, H, K, V), "S", false);
+    // the sketch's tensors too, before S is touched (the flush below checks them again)
+    const bool any_sketch = p->rtot > 0;
+    CHECK_T(omega, any_sketch ? fbytes(d.groups, d.basis_rows, K) : 0, "omega", !any_sketch);
+    CHECK_T(Y, any_sketch ? fbytes(B, p->rtot, V) : 0, "Y", !any_sketch);
     if (toks) {
         sk::PrefillArgs A;
         A.kind = d.kind;

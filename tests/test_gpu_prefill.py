@@ -104,3 +104,19 @@ def test_prefill_rejects_a_negative_length():
         rs.sketchssm_prefill(gpu.plan, -1, None, None, None, None, gpu.S, gpu.omega, gpu.Y)
     torch.cuda.synchronize()
     gpu.close()
+
+
+def test_prefill_refused_before_the_state_is_touched():
+    """A missing basis (the layer has sketch heads) is refused before the prompt is
+    applied: S keeps its values."""
+    import torch
+    import rank_state_read_b200 as rs
+    cfg = synth.config(0).replace(B=2)
+    gpu = make_layer(cfg, synth.layer_rank_table(cfg), synth.basis(cfg), synth.init_state(cfg, range(cfg.B)))
+    d = to_dev(synth.prompt_inputs(cfg, 5, range(cfg.B)))
+    S_before = gpu.S.clone()
+    with pytest.raises(rs.SketchSSMError):
+        rs.sketchssm_prefill(gpu.plan, 5, d["k"], d["v"], d["a"], d["beta"], gpu.S, None, gpu.Y)
+    torch.cuda.synchronize()
+    assert torch.equal(gpu.S, S_before)
+    gpu.close()
