@@ -1,0 +1,52 @@
+"""bench.py's algorithmic counts (the numerators of its roofline fractions) against
+figures worked out by hand from the layer shapes (CPU only).
+
+Per decode step and batch row the sketch decode moves the sketch rows of the sketch
+heads, the state of the dense heads, q, the step's token twice (read, then appended),
+the buffered tokens (7.5 on average over a window) and y; the dense-read decode moves
+the whole state instead of the sketch rows.  Worked out for the Mamba-2 layer at batch
+256 (sum of ranks 762, one dense head), the GDN layer at batch 512 and the KDA layer
+at batch 1024, these come to 195 / 1465 MB, 276 / 1251 MB and 743 / 2660 MB a step;
+the Mamba-2 flush of 16 tokens to 2.93 GB.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import bench
+import synth
+
+HAND = {  # config: (sketch decode MB, dense-read decode MB), mean over the window
+    1: (195, 1465),
+    3: (276, 1251),
+    4: (743, 2660),
+}
+
+
+@pytest.mark.parametrize("cid", sorted(HAND))
+def test_decode_bytes_match_the_hand_figures(cid):
+    cfg = synth.config(cid)
+    rank = synth.layer_rank_table(cfg)
+    sk = np.mean([bench.decode_bytes(cfg, rank, p) for p in range(cfg.W)]) / 1e6
+    dn = np.mean([bench.dense_decode_bytes(cfg, p) for p in range(cfg.W)]) / 1e6
+    assert abs(sk - HAND[cid][0]) / HAND[cid][0] < 5e-3
+    assert abs(dn - HAND[cid][1]) / HAND[cid][1] < 5e-3
+
+
+def test_flush_and_step_bytes_of_the_mamba2_layer():
+    cfg = synth.config(1)
+    rank = synth.layer_rank_table(cfg)
+    assert abs(bench.flush_bytes(cfg, rank, cfg.W) / 1e9 - 2.93) < 0.01
+    # the standard step moves the state twice: 2 x 256 x 128 x 128 x 80 x 4 bytes, plus
+    # the token (q, k, v, a) and y
+    state = 2 * 256 * 128 * 128 * 80 * 4
+    extra = 256 * 4 * (2 * 8 * 128 + 2 * 128 * 80 + 128)
+    assert bench.step_bytes(cfg) == state + extra
+
+
+def test_prefill_instruction_counts():
+    """One FMA per state element and token (Mamba-2), two (GDN), three (KDA)."""
+    for cid, per in ((1, 1), (3, 2), (4, 3)):
+        cfg = synth.config(cid)
+        assert bench.prefill_instr(cfg, 64) == per * cfg.B * cfg.H * cfg.K * cfg.V * 64
