@@ -216,12 +216,23 @@ def oracle_cycles(cfg, rank, omega, rows, min_s: float, max_cycles: int):
 
 
 def cpu_baseline(cfg, rank, omega) -> dict:
+    """The oracle on every host core over the whole batch (about 10 s), then on one
+    core over 8 batch rows (about 4 s; rows are independent, so tok/s compares)."""
+    import oracle
     rows = list(range(cfg.B))
     cycles, el, threads = oracle_cycles(cfg, rank, omega, rows, min_s=10.0, max_cycles=64)
     tok = cfg.B * cfg.W * cycles
+    oracle.set_num_threads(1)
+    try:
+        rows1 = rows[:8]
+        c1, el1, _ = oracle_cycles(cfg, rank, omega, rows1, min_s=4.0, max_cycles=64)
+    finally:
+        oracle.set_num_threads(threads)
     return {"value": tok / el, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{cycles} window cycle(s) ({cycles * cfg.W} decode steps + {cycles} flushes) "
-                      f"of one layer at batch {cfg.B}, fp64, {el:.1f} s"}
+                      f"of one layer at batch {cfg.B}, fp64, {el:.1f} s",
+            "value_1_core": len(rows1) * cfg.W * c1 / el1,
+            "sample_1_core": f"{c1} window cycle(s) of {len(rows1)} batch rows on one core, {el1:.1f} s"}
 
 
 # ----------------------------------------------------------------------------- ranks

@@ -15,4 +15,5 @@ Parity is pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py``;
 nothing here is "parity unpinned" except the accuracy of a rank-r sketch against the
 exact read on real models (that needs a calibrated basis the pages do not publish).
 """
-from .core import OracleLayer, layout, load_library, num_threads, prefill, standard_step, trajectory  # noqa: F401
+from .core import (OracleLayer, layout, load_library, num_threads, prefill, set_num_threads,  # noqa: F401
+                   standard_step, trajectory)

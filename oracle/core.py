@@ -43,12 +43,19 @@ def _load():
         lib.oracle_prefill.restype = None
         lib.oracle_prefill.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int32, P, P, P, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.restype = None
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
     return _lib
 
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Host threads of the oracle's loops from now on."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def _p(a: Optional[np.ndarray]):

@@ -314,6 +314,17 @@ void oracle_prefill(const oracle_dims *d, int32_t T, double *S, const double *pk
     }
 }
 
+/* Host threads the loops above use from now on (a single-thread baseline sets 1). */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    omp_set_num_threads(n < 1 ? 1 : n);
+#else
+    (void)n;
+#endif
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP
