@@ -46,7 +46,9 @@
  *    sketchssm_decode(pos) appends the step's token at buffer slot pos and returns
  *    y including it.  After the decode at pos = W-1 the caller runs
  *    sketchssm_flush(n_tokens = W) and restarts at pos = 0.  sketchssm_flush with
- *    n_tokens = 0 forms the sketch of an initial state.
+ *    n_tokens = 0 forms the sketch of an initial state; sketchssm_prefill applies a
+ *    prompt to the state and then forms its sketch, after which decoding starts at
+ *    pos = 0.
  *  - Supported shapes: K = 128, V a multiple of 16 in [16, 256], 1 <= W <= 32,
  *    H divisible by G with H/G <= 32, Hqk dividing H and divisible by G,
  *    1 <= rank_cap <= basis_rows <= K.  Others return SKETCHSSM_ERR_UNSUPPORTED.
