@@ -539,3 +539,34 @@ def test_prefill_mutations_are_caught(name, old, new, kind, tmp_path):
     cfg = tiny_cfg(kind, Hqk=2 if kind == "mamba2" else None)
     rank = np.array([1, DENSE, 2, 3], np.int32)
     assert check_handoff_against_brute(cfg, rank, T=2 * cfg.W, lib=lib) > 1e-6
+
+
+# --------------------------------------------------------------------------- projected exact read
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+def test_sketch_read_is_the_exact_read_of_the_projected_state(kind):
+    """Right after a flush and at every later position of the window, a sketch head's
+    output equals the exact output of the layer whose flushed state of that head is
+    replaced by its projection P S_f (P = Omega_r^T Omega_r): the sketch only ever
+    stands in for S_f, and the buffered tokens are replayed exactly.  Dense heads are
+    read exactly in both."""
+    cfg = tiny_cfg(kind, K=8, V=5, W=4, Hqk=2 if kind == "mamba2" else None)
+    rank = np.array([3, DENSE, 1, 5], np.int32)
+    rows = list(range(cfg.B))
+    omega = synth.basis_fp64(cfg)
+    S0 = synth.init_state(cfg, rows).astype(np.float64)
+    Sp = S0.copy()
+    for h in range(cfg.H):
+        if rank[h] != DENSE:
+            O = omega[h * cfg.G // cfg.H, :rank[h]]
+            Sp[:, h] = np.einsum("kl,blv->bkv", O.T @ O, S0[:, h])
+    mk = lambda S: oracle.OracleLayer(kind, H=cfg.H, Hqk=cfg.Hqk, K=cfg.K, V=cfg.V, W=cfg.W, G=cfg.G,
+                                      rank=rank, omega=omega, S0=S)
+    sk, ex = mk(S0), mk(Sp)
+    sk.flush(0)
+    ex.flush(0)
+    for t in range(cfg.W):
+        inp = synth.step_inputs(cfg, t, rows)
+        ys = sk.decode(t, inp)
+        ye = ex.decode(t, inp, dense_all=True)
+        assert rel(ys, ye) < 1e-12, t
