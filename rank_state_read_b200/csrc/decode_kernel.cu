@@ -12,11 +12,11 @@
 // value rows.  The step splits into
 //
 //  1. the query-side products, written to the plan's scratch:
-//     Mamba-2 (dots_kernel_mamba2), one CTA per (q/k head, up to 8 batch rows): the
+//     Mamba-2 (dots_kernel_mamba2), one CTA per (q/k head, 4 batch rows): the
 //       group's basis rows, the rows' queries and buffered keys are staged in shared
-//       memory in one round; s_i = k_i . q (one lane per key) and
-//       u_m = Omega_g[m] . q (register-blocked over the CTA's rows) are written per
-//       (batch row, q/k head).  The step's key is appended to buffer slot pos.
+//       memory by one round of cp.async; every product s_i = k_i . q and
+//       u_m = Omega_g[m] . q is then one thread's loop over 128 staged floats, written
+//       per (batch row, q/k head).  The step's key is appended to buffer slot pos.
 //     GDN/KDA (coef_kernel_delta), one warp per (batch row, head): walk the buffer
 //       newest first, x <- M_i^T x, keys (and KDA decays) prefetched four steps
 //       ahead; the replay coefficients beta_i (k_i . x) and the base coefficients
