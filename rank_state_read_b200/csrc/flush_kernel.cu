@@ -21,7 +21,7 @@
 //   hi hi + hi lo + lo hi, which keeps fp32 accuracy); the state lives in the
 //   accumulator layout (columns 8 nt + 2 t (+1) for lane 4 g + t, and a fixed map of
 //   accumulator rows to state rows that keeps the fragment reads of the padded 4-row
-//   chunks conflict-free).  Key and value rows are staged with 8 floats of padding.
+//   chunks conflict-free).  Staged value rows carry 8 floats of padding, key rows 4.
 //   GDN / KDA: thread (ks, c4) holds the float4 column chunk c4 of the 16 state rows
 //   4 ks + 32 q + e (q, e < 4) and applies the delta rule token by token; every
 //   reduction over k stays inside the warp, and the float4 reads of keys and decays by
