@@ -81,3 +81,21 @@ def test_step_inputs_distributions_and_row_independence():
         one = synth.step_inputs(cfg, 5, [2])
         for x in ("q", "k", "v", "a"):
             assert np.array_equal(one[x][0], s[x][2])
+
+
+def test_prompt_rows_regenerate_alone_and_follow_the_step_distributions():
+    """Every (row, token) of a prompt has its own stream: a subset of rows regenerates
+    exactly; keys are unit vectors, decays lie in (0, 1), beta only for GDN / KDA."""
+    for cid in (1, 3, 4):
+        cfg = synth.config(cid)
+        full = synth.prompt_inputs(cfg, 5, range(4))
+        part = synth.prompt_inputs(cfg, 5, [2])
+        for key in ("k", "v", "a"):
+            assert np.array_equal(full[key][2:3], part[key])
+        assert (full["beta"] is None) == (cfg.kind == "mamba2")
+        assert np.allclose(np.linalg.norm(full["k"].astype(np.float64), axis=-1), 1.0, atol=1e-6)
+        assert (full["a"] > 0).all() and (full["a"] < 1).all()
+        assert full["k"].shape == (4, 5, cfg.Hqk, cfg.K) and full["v"].shape == (4, 5, cfg.H, cfg.V)
+        # a prompt's tokens are not the decode steps' tokens
+        step0 = synth.step_inputs(cfg, 0, range(4))
+        assert not np.array_equal(full["v"][:, 0], step0["v"])
