@@ -111,6 +111,12 @@ def flush_bytes(cfg, rank, n: int) -> int:
     return cfg.B * row + omega_bytes(cfg, rank)
 
 
+def decode_launches(cfg) -> int:
+    """Kernel launches of one sketch-decode call: the one-launch form for Mamba-2, the
+    coefficient kernel and the combine for GDN / KDA."""
+    return 1 if cfg.kind == "mamba2" else 2
+
+
 # ----------------------------------------------------------------------------- environment
 
 def hbm_peak():
@@ -337,8 +343,8 @@ def run_ours(args, cfg) -> None:
     ms = t_start.elapsed_time(t_end)
     dec = [(p, a.elapsed_time(b)) for p, a, b in ev["decode"]]
     fl = [b_.elapsed_time(c_) for _, b_, c_ in ev["flush"]]
-    # every decode call is two launches (the products kernel and the combine kernel)
-    launches = 2 * len(ev["decode"]) + len(ev["flush"])
+    # a Mamba-2 sketch decode is one launch; GDN / KDA: the coefficient kernel + the combine
+    launches = decode_launches(cfg) * len(ev["decode"]) + len(ev["flush"])
 
     # ---- dense-read baseline decode (same positions, same replicas)
     kd = max(1, min(args.steps, 10))

@@ -114,9 +114,18 @@ typedef void *sketchssm_stream;
  * the host knows Rtot and the item counts.  *out is set only on success.
  * Source: the calibration stage "allocate" of the sketchssm PyPI page (each head
  * gets a rank or falls back to dense) and its stage "basis" (one basis per group).
+ *
+ * group_host: the basis group of every head (host, [H] int32, values 0..G-1), or NULL
+ * for the layout the kernels are built for: contiguous runs of H/G heads, head h in
+ * group h / (H/G) (Mamba-2's heads of one B/C group sit side by side).  A table equal to
+ * that layout is accepted; any other map returns SKETCHSSM_ERR_UNSUPPORTED (a value
+ * outside 0..G-1: SKETCHSSM_ERR_INVALID_ARG).  Heads are independent on this path, so a
+ * caller whose groups interleave numbers its heads group by group (permuting the head
+ * axis of its q/k/v/a/beta/S tensors and the rank table alike) and gets the same result.
  */
 sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t *rank_host,
-                                       sketchssm_stream stream, sketchssm_plan **out);
+                                       const int32_t *group_host, sketchssm_stream stream,
+                                       sketchssm_plan **out);
 
 /*
  * Copy the plan's layout tables to host memory (reads host copies; no GPU work).
@@ -172,9 +181,9 @@ sketchssm_status sketchssm_flush(const sketchssm_plan *plan, float *S, const flo
                                  sketchssm_stream stream);
 
 /*
- * Sketch decode (read-sketch step; paper abstract: "combines the sketch vectors
- * with query-dependent coefficients to reconstruct the output without a full-state
- * read").  pos in [0, W): tokens buffered since the last flush.  Appends the step's
+ * Sketch decode (read-sketch step; SketchSSM, Abstract: the output of a decode step is
+ * rebuilt from the sketch rows weighted by coefficients taken from the query, and the
+ * full state is not read).  pos in [0, W): tokens buffered since the last flush.  Appends the step's
  * token (k, v, a, beta) at buffer slot pos, then for every (b, h) with n = pos+1:
  *   replay: walk the buffered tokens newest first with x = q,
  *           y += beta_i (k_i . x) v_i,  x <- M_i^T x;      q0 = final x
@@ -192,8 +201,9 @@ sketchssm_status sketchssm_decode(const sketchssm_plan *plan, int32_t pos, const
                                   const float *S, float *y, sketchssm_stream stream);
 
 /*
- * Dense-read decode: the ReplaySSM baseline the paper improves on ("each new query
- * still requires a full-state read").  Same as sketchssm_decode, but every head
+ * Dense-read decode: the ReplaySSM baseline the paper improves on (SketchSSM, Abstract:
+ * with buffered updates alone, every query still reads the whole state).  Same as
+ * sketchssm_decode, but every head
  * reads S exactly (y += S_h^T q0) whatever its rank.  Reads S, never Y or omega.
  */
 sketchssm_status sketchssm_dense_decode(const sketchssm_plan *plan, int32_t pos, const float *q,
@@ -205,7 +215,10 @@ sketchssm_status sketchssm_dense_decode(const sketchssm_plan *plan, int32_t pos,
 /*
  * Sketch decode whose scratch comes from a fixed static device array instead of the
  * plan's buffer; the paper has no counterpart (it is a memory-ownership variant of
- * sketchssm_decode, with the same arguments, layouts and results).
+ * sketchssm_decode, with the same arguments and layouts).  It runs the two-launch form
+ * of the decode (products, then combine), whose products pass through scratch; its
+ * results equal sketchssm_decode's up to fp32 rounding (for Mamba-2, sketchssm_decode
+ * runs the one-launch form, which sums the same terms in another order).
  *
  * For callers that must not allocate device memory at all once serving has started:
  * an engine that has handed every free byte of HBM to its own state and KV pools, so
@@ -218,9 +231,10 @@ sketchssm_status sketchssm_dense_decode(const sketchssm_plan *plan, int32_t pos,
  *    (Mamba-2: batch * qk_heads * round4(window + rank_cap) floats; GDN / KDA: batch
  *    * the plan's coefficient floats per batch row) returns SKETCHSSM_ERR_INVALID_ARG
  *    with the sizes in sketchssm_last_error(), before any tensor is looked at.
- *  - Set-up: the first call on a device looks the array's address up there (with that
- *    device current, which the plan check already requires); make that first call
- *    before any stream capture.  Later calls only read the cached address.
+ *  - Set-up: every call looks the array's address up on the current device (the plan
+ *    check already requires the plan's device to be current); the lookup allocates
+ *    nothing.  The first lookup on a device may load the library's device code there,
+ *    so make the first call on each device before any stream capture.
  *  - Sharing: every call on a device, from every plan and host thread, uses the same
  *    array.  Calls whose kernels overlap on the GPU (different streams without an
  *    ordering between them) race on it and give wrong results; calls in stream order

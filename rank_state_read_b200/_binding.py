@@ -52,7 +52,7 @@ def load():
                            "(nvcc, sm_100a); there is no fallback implementation")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
-    lib.sketchssm_plan_create.argtypes = [ctypes.POINTER(Desc), P, P, ctypes.POINTER(P)]
+    lib.sketchssm_plan_create.argtypes = [ctypes.POINTER(Desc), P, P, P, ctypes.POINTER(P)]
     lib.sketchssm_plan_query.argtypes = [P, ctypes.POINTER(I64), P, P, I32, P, ctypes.POINTER(I32)]
     lib.sketchssm_plan_check.argtypes = [P, P]
     lib.sketchssm_plan_set_wait_limit.argtypes = [P, I64]
@@ -109,7 +109,7 @@ class Plan:
 
     def __init__(self, kind: str, *, batch: int, heads: int, qk_heads: int, key_dim: int,
                  value_dim: int, window: int, groups: int, basis_rows: int, rank_cap: int,
-                 rank: Sequence[int], stream=None):
+                 rank: Sequence[int], group: Optional[Sequence[int]] = None, stream=None):
         lib = load()
         self.kind = kind
         self.desc = Desc(KINDS[kind], batch, heads, qk_heads, key_dim, value_dim, window, groups,
@@ -117,8 +117,14 @@ class Plan:
         if len(rank) != heads:
             raise ValueError("rank table must have one entry per head")
         rank_arr = (ctypes.c_int32 * heads)(*[int(r) for r in rank])
+        group_arr = None
+        if group is not None:
+            if len(group) != heads:
+                raise ValueError("group table must have one entry per head")
+            group_arr = (ctypes.c_int32 * heads)(*[int(g) for g in group])
         handle = ctypes.c_void_p()
         _check(lib.sketchssm_plan_create(ctypes.byref(self.desc), ctypes.cast(rank_arr, ctypes.c_void_p),
+                                         None if group_arr is None else ctypes.cast(group_arr, ctypes.c_void_p),
                                          _stream(stream), ctypes.byref(handle)), "sketchssm_plan_create")
         self.handle = handle
         self.rank = [int(r) for r in rank]

@@ -443,7 +443,12 @@ combine_kernel(const DecodeArgs A)
     if (__syncthreads_or(!ok)) {
         if (tid == 0) atomicOr(A.status, SK_STATUS_DECODE_TIMEOUT);
         ok = mbar_wait_bounded(bar, 0, DEFAULT_WAIT_CYCLES);
-        if (__syncthreads_or(!ok)) return;
+        if (__syncthreads_or(!ok)) {
+            // give up: let the copies still in flight land (bounded) before the CTA exits
+            if (tid == 0) mbar_wait_bounded(bar, 0, DEFAULT_WAIT_CYCLES);
+            __syncthreads();
+            return;
+        }
     }
     const int V4 = V >> 2;
     for (int o = tid; o < nh * V4; o += blockDim.x) {

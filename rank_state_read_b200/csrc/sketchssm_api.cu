@@ -6,7 +6,6 @@
 
 #include <cstdio>
 #include <cstring>
-#include <mutex>
 #include <string>
 
 #include "internal.cuh"
@@ -229,7 +228,8 @@ const char *sketchssm_status_string(sketchssm_status s)
 const char *sketchssm_last_error(void) { return g_last_error.c_str(); }
 
 sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t *rank_host,
-                                       sketchssm_stream stream, sketchssm_plan **out)
+                                       const int32_t *group_host, sketchssm_stream stream,
+                                       sketchssm_plan **out)
 {
     g_last_error.clear();
     if (!out) return fail(SKETCHSSM_ERR_INVALID_ARG, "out is NULL");
@@ -238,6 +238,21 @@ sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t
     if (!rank_host) return fail(SKETCHSSM_ERR_INVALID_ARG, "rank table is NULL");
     const sketchssm_desc d = *desc;
     const int H = d.heads, G = d.groups;
+    if (group_host) {
+        // the kernels are built for contiguous groups of H/G heads
+        for (int h = 0; h < H; ++h) {
+            const int g = group_host[h];
+            if (g < 0 || g >= G)
+                return fail(SKETCHSSM_ERR_INVALID_ARG, "group[" + std::to_string(h) + "] = " + std::to_string(g) +
+                                                           " is outside [0, groups)");
+        }
+        for (int h = 0; h < H; ++h)
+            if (group_host[h] != h / (H / G))
+                return fail(SKETCHSSM_ERR_UNSUPPORTED,
+                            "group[" + std::to_string(h) + "] = " + std::to_string(group_host[h]) +
+                                ": only contiguous groups (head h in group h / (heads / groups)) are supported; "
+                                "number the heads group by group");
+    }
     long long rtot = 0;
     for (int h = 0; h < H; ++h) {
         const int r = rank_host[h];
@@ -504,7 +519,8 @@ sketchssm_status sketchssm_decode_rows(const sketchssm_plan *p, const int32_t *p
     int most = 0;
     for (int c : p->h_items) most = c > most ? c : most;
     A.n_items = most;
-    cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
+    cudaError_t e = sk::decode_group_supported(A) ? sk::launch_decode_group(A, (cudaStream_t)stream)
+                                                  : sk::launch_decode(A, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     return SKETCHSSM_OK;
 }
@@ -525,7 +541,8 @@ sketchssm_status sketchssm_decode(const sketchssm_plan *p, int32_t pos, const fl
     CHECK_T(omega, any_sketch ? fbytes(d.groups, d.basis_rows, d.key_dim) : 0, "omega", !any_sketch);
     CHECK_T(S, any_dense ? fbytes(d.batch, d.heads, d.key_dim, d.value_dim) : 0, "S", !any_dense);
     const sk::DecodeArgs A = decode_args(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, Y, omega, S, y, 0);
-    cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
+    cudaError_t e = sk::decode_group_supported(A) ? sk::launch_decode_group(A, (cudaStream_t)stream)
+                                                  : sk::launch_decode(A, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     return SKETCHSSM_OK;
 }
@@ -567,24 +584,16 @@ static __device__ __align__(256) float g_static_scratch[SKETCHSSM_STATIC_SCRATCH
 
 namespace {
 
-constexpr int STATIC_SCRATCH_DEVICES = 64;
-std::mutex g_static_mu;
-float *g_static_ptr[STATIC_SCRATCH_DEVICES];  // address of the array on each device
-
-// The array's address on device `dev`, which must be current.  Looked up by the first
-// call on that device, cached afterwards.
-sketchssm_status static_scratch(int dev, float **out)
+// The array's address on the current device.  Looked up on every call: the lookup
+// allocates nothing, and a cached address would go stale if the device's context were
+// destroyed and created again (cudaDeviceReset), which reloads the library's device code.
+// The first lookup on a device may load that code there.
+sketchssm_status static_scratch(float **out)
 {
-    if (dev < 0 || dev >= STATIC_SCRATCH_DEVICES)
-        return fail(SKETCHSSM_ERR_UNSUPPORTED, "static scratch: device ordinal above 63");
-    std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_ptr[dev]) {
-        void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
-        g_static_ptr[dev] = static_cast<float *>(p);
-    }
-    *out = g_static_ptr[dev];
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    *out = static_cast<float *>(p);
     return SKETCHSSM_OK;
 }
 
@@ -623,7 +632,7 @@ extern "C" sketchssm_status sketchssm_decode_static_scratch(const sketchssm_plan
     CHECK_T(omega, any_sketch ? fbytes(d.groups, d.basis_rows, d.key_dim) : 0, "omega", !any_sketch);
     CHECK_T(S, any_dense ? fbytes(d.batch, d.heads, d.key_dim, d.value_dim) : 0, "S", !any_dense);
     float *scratch = nullptr;
-    if ((s = static_scratch(p->device, &scratch)) != SKETCHSSM_OK) return s;
+    if ((s = static_scratch(&scratch)) != SKETCHSSM_OK) return s;
     sk::DecodeArgs A = decode_args(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, Y, omega, S, y, 0);
     A.scratch = scratch;
     cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);

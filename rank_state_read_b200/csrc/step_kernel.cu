@@ -104,7 +104,12 @@ __global__ void __launch_bounds__(STEP_MAXT, KIND == SKETCHSSM_MAMBA2 ? 4 : 3) s
     if (__syncthreads_or(!ok)) {
         if (tid == 0) atomicOr(A.status, SK_STATUS_STEP_TIMEOUT);
         ok = mbar_wait_bounded(bar, 0, DEFAULT_WAIT_CYCLES);
-        if (__syncthreads_or(!ok)) return;
+        if (__syncthreads_or(!ok)) {
+            // give up: let the copies still in flight land (bounded) before the CTA exits
+            if (tid == 0) mbar_wait_bounded(bar, 0, DEFAULT_WAIT_CYCLES);
+            __syncthreads();
+            return;
+        }
     }
 
     float4 s[16];

@@ -15,3 +15,12 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def root():
     return ROOT
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With PARITY_REPORT=<path> set, write the error records of every parity run of the
+    session (rel, per-head and element-wise measures; see gpu_util) to that file."""
+    path = os.environ.get("PARITY_REPORT")
+    mod = sys.modules.get("gpu_util")
+    if path and mod is not None and mod.REPORT:
+        mod.write_report(path)

@@ -46,11 +46,13 @@ def test_status_strings(lib):
 def _create(lib, **over):
     d = dict(kind=0, batch=4, heads=8, qk_heads=1, key_dim=128, value_dim=80, window=16, groups=1,
              basis_rows=128, rank_cap=128)
-    d.update(over)
+    d.update({k: v for k, v in over.items() if k != "group_table"})
     desc = rs.Desc(*[d[f] for f, _ in rs.Desc._fields_])
     ranks = (ctypes.c_int32 * d["heads"])(*([6] * d["heads"]))
     out = ctypes.c_void_p()
-    st = lib.sketchssm_plan_create(ctypes.byref(desc), ctypes.cast(ranks, ctypes.c_void_p), None,
+    group = over.get("group_table")
+    gp = None if group is None else ctypes.cast((ctypes.c_int32 * d["heads"])(*group), ctypes.c_void_p)
+    st = lib.sketchssm_plan_create(ctypes.byref(desc), ctypes.cast(ranks, ctypes.c_void_p), gp, None,
                                    ctypes.byref(out))
     return st, out, lib.sketchssm_last_error().decode()
 
@@ -73,12 +75,28 @@ def test_plan_create_rejects_bad_ranks(lib):
     out = ctypes.c_void_p()
     for bad in ([6, 0, 6, 6], [6, 50, 6, 6], [6, -2, 6, 6]):
         ranks = (ctypes.c_int32 * 4)(*bad)
-        st = lib.sketchssm_plan_create(ctypes.byref(desc), ctypes.cast(ranks, ctypes.c_void_p), None,
+        st = lib.sketchssm_plan_create(ctypes.byref(desc), ctypes.cast(ranks, ctypes.c_void_p), None, None,
                                        ctypes.byref(out))
         assert st == 1 and not out.value
         assert b"rank[1]" in lib.sketchssm_last_error()
-    assert lib.sketchssm_plan_create(ctypes.byref(desc), None, None, ctypes.byref(out)) == 1
-    assert lib.sketchssm_plan_create(None, None, None, ctypes.byref(out)) == 1
+    assert lib.sketchssm_plan_create(ctypes.byref(desc), None, None, None, ctypes.byref(out)) == 1
+    assert lib.sketchssm_plan_create(None, None, None, None, ctypes.byref(out)) == 1
+
+
+@pytest.mark.parametrize("group,status", [
+    ([0, 0, 1, 1, 2, 2, 3, 3][::-1], 3),   # groups in reverse order
+    ([0, 1, 0, 1, 2, 3, 2, 3], 3),         # interleaved
+    ([0, 0, 0, 1, 1, 2, 3, 3], 3),         # unequal runs
+    ([0, 0, 1, 1, 2, 2, 3, 4], 1),         # a group outside 0..G-1
+    ([0, 0, 1, 1, 2, 2, -1, 3], 1),
+])
+def test_plan_create_group_table_checked_on_the_host(lib, group, status):
+    """Only the contiguous head-to-group map is supported; any other is refused before
+    anything is allocated or launched, with the offending head named."""
+    st, out, msg = _create(lib, heads=8, groups=4, qk_heads=4, group_table=group)
+    assert st == status, msg
+    assert not out.value
+    assert "group[" in msg
 
 
 def test_calls_without_a_plan(lib):

@@ -112,6 +112,21 @@ def test_layout_bit_exact(name, cfg, rank):
     plan.close()
 
 
+def test_layout_with_explicit_contiguous_group_table():
+    """A group table equal to the contiguous layout is accepted and gives the same
+    tables as NULL."""
+    import rank_state_read_b200 as rs
+    cfg = synth.config(1)
+    rank = synth.layer_rank_table(cfg)
+    kw = dict(batch=1, heads=cfg.H, qk_heads=cfg.Hqk, key_dim=cfg.K, value_dim=cfg.V, window=cfg.W,
+              groups=cfg.G, basis_rows=cfg.Rb, rank_cap=cfg.cap, rank=rank.tolist())
+    a = rs.Plan(cfg.kind, **kw)
+    b = rs.Plan(cfg.kind, group=[h // (cfg.H // cfg.G) for h in range(cfg.H)], **kw)
+    assert (a.offsets, a.rmax, a.r_total, a.work) == (b.offsets, b.rmax, b.r_total, b.work)
+    a.close()
+    b.close()
+
+
 # ----------------------------------------------------------------------------- small, every row
 
 def test_config0_full_trajectory():
@@ -178,6 +193,18 @@ def test_other_shapes(V, W, H, G):
     parity_run(cfg, 2 * W + 3)
 
 
+MAMBA2_SHAPES = [(16, 5, 8, 2, 2), (48, 7, 64, 2, 64), (256, 8, 4, 1, 1), (128, 1, 32, 1, 1),
+                 (256, 4, 32, 1, 32), (80, 32, 32, 2, 2)]
+
+
+@pytest.mark.parametrize("V,W,H,G,Hqk", MAMBA2_SHAPES)
+def test_other_shapes_mamba2(V, W, H, G, Hqk):
+    """Mamba-2 at other value dims, windows and group sizes (up to 32 heads and 256
+    columns per group, the largest one-launch CTA), q/k shared by a group or per head."""
+    cfg = small(1, B=3, V=V, W=W, H=H, G=G, Hqk=Hqk, n_dense=1)
+    parity_run(cfg, 2 * W + 3)
+
+
 @pytest.mark.parametrize("cid", [1, 3, 4])
 def test_ring_reuse_moderate_batch(cid):
     """Enough batch rows that every persistent decode CTA walks several units through
@@ -190,32 +217,53 @@ def test_single_row_batch():
     parity_run(small(1, B=1), 17)
 
 
-# ----------------------------------------------------------------------------- full size, sampled rows
+# ----------------------------------------------------------------------------- full size, every row
 
 FULL = [(1, 20), (3, 18), (4, 17)]
 
 
 @pytest.mark.parametrize("cid,T", FULL, ids=[f"config{c}" for c, _ in FULL])
-def test_full_size_sampled_rows(cid, T):
-    """The workloads at their full batch, in the bench's launch configuration; the
-    oracle computes a seeded sample of batch rows (rows are independent)."""
-    cfg = synth.config(cid)
-    rng = np.random.default_rng(cid)
-    rows = sorted({0, 1, cfg.B // 2, cfg.B - 1, *rng.integers(0, cfg.B, 3).tolist()})
-    parity_run(cfg, T, rows=rows)
+def test_full_size_all_rows(cid, T):
+    """The workloads at their full batch, in the bench's launch configuration, every
+    batch row against the oracle (a flush of 16 tokens and the steps after it)."""
+    parity_run(synth.config(cid), T, name=f"full-config{cid}")
 
 
 @pytest.mark.parametrize("cid", [1, 3])
-def test_full_size_dense_read_sampled_rows(cid):
-    cfg = synth.config(cid)
-    parity_run(cfg, 17, rows=[0, cfg.B // 3, cfg.B - 1], dense=True)
+def test_full_size_dense_read_all_rows(cid):
+    parity_run(synth.config(cid), 17, dense=True, name=f"full-dense-read-config{cid}")
 
 
-@pytest.mark.parametrize("m", [4, 21])
-def test_stack_layer_sampled_rows(m):
-    """One layer of the 27-layer stack sweep (its own rank table: up to 22% dense)."""
-    cfg = synth.config(2, mean_rank=m, batch=256)
+def test_full_size_per_head_qk_mamba2_sampled_rows():
+    """The Mamba-2 layer with q/k per head (the layer's secondary q/k layout)."""
+    cfg = synth.config(1).replace(Hqk=128)
+    parity_run(cfg, 17, rows=[0, 1, 77, 128, 255], name="full-config1-per-head-qk")
+
+
+# ----------------------------------------------------------------------------- the 27-layer stack sweep
+
+STACK_POINTS = [(m, B) for m in (4, 6, 10, 21) for B in (64, 256, 1024)]
+
+
+def stack_layers(table):
+    """The layer with the most dense heads and the one with the fewest (ties: first)."""
+    nd = (table == DENSE).sum(axis=1)
+    return int(np.argmax(nd)), int(np.argmin(nd))
+
+
+@pytest.mark.parametrize("m,B", STACK_POINTS, ids=[f"r{m}-b{B}" for m, B in STACK_POINTS])
+def test_stack_sweep_point(m, B):
+    """Every point of the stack sweep (mean rank x batch): the most-dense and the
+    least-dense layer of the point's rank tables, each with its own basis and inputs.
+    Every row at batch 64 and 256; at batch 1024 a seeded sample of 64 rows (the
+    others run on the GPU with states drawn on the device)."""
+    cfg = synth.config(2, mean_rank=m, batch=B)
     table = synth.stack_rank_tables(cfg)
-    layer = int(np.argmax((table == DENSE).sum(axis=1)))
     one = cfg.replace(layers=1)
-    parity_run(one, 17, rank=table[layer], rows=[0, 100, 255])
+    rows = None
+    if B > 256:
+        rng = np.random.default_rng(1000 * m + B)
+        rows = sorted({0, B - 1, *rng.choice(B, 62, replace=False).tolist()})
+    for layer in sorted(set(stack_layers(table))):
+        parity_run(one, 17, rank=table[layer], rows=rows, layer=layer,
+                   init="numpy" if rows is None else "sampled", name=f"stack-r{m}-b{B}-layer{layer}")

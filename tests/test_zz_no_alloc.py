@@ -1,16 +1,24 @@
 """sketchssm_decode_static_scratch (the decode whose scratch is the library's static
-device array) against sketchssm_decode (the plan's own scratch) on the same inputs.
+device array) against sketchssm_decode on the same inputs.
 
-The two run the same kernels on the same data, so y and the appended buffers must be
-identical bit for bit.  Two decode calls in a row on the static path check that the
-second call does not depend on what the first left in the shared array.  This file is
-collected last so that it also runs after every other GPU test in the session.
+It serves callers that cannot allocate device memory once they are serving (an engine
+that has given all free HBM to its own pools, or code that must not take cudaMalloc's
+implicit synchronisation); nothing in the call allocates.  The static call runs the
+two-launch decode (products through scratch, then the combine); sketchssm_decode runs
+the same two launches for GDN / KDA and, for Mamba-2, the one-launch decode, which
+sums the same terms in another order.  So y must agree within the parity tolerance
+(max |diff| / max |ref| <= 1e-4, the bar of every parity test), and bit for bit where
+both calls run the same kernels; the appended buffers are copies and agree bit for bit.
+Two decode calls in a row on the static path check that the second call does not
+depend on what the first left in the shared array.  This file is collected last so
+that it also runs after every other GPU test in the session.
 """
 from __future__ import annotations
 
 import pytest
 
 import synth
+from gpu_util import TOL, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -36,6 +44,13 @@ def _static_decode(layer, pos, x, y):
     rs.sketchssm_decode_static_scratch(layer.plan, pos, x["q"], x["k"], x["v"], x["a"], x["beta"],
                                        layer.kbuf, layer.vbuf, layer.abuf, layer.bbuf, layer.Y,
                                        layer.omega, layer.S, y)
+
+
+def _same_y(kind, y_sta, y_ref):
+    import torch
+    if kind != "mamba2":
+        return torch.equal(y_sta, y_ref)
+    return bool(torch.isfinite(y_sta).all()) and rel_err(y_sta.cpu().numpy(), y_ref.cpu().numpy()) <= TOL
 
 
 def _buffers(layer):
@@ -66,7 +81,7 @@ def test_two_calls_in_a_row_match_plan_scratch(cid, B):
         y_sta = torch.full_like(y_ref, float("nan"))
         _static_decode(sta, pos, x, y_sta)
         torch.cuda.synchronize()
-        assert torch.equal(y_sta, y_ref), f"y differs at pos {pos}"
+        assert _same_y(cfg.kind, y_sta, y_ref), f"y differs at pos {pos}"
         for a, b in zip(_buffers(sta), _buffers(ref)):
             assert torch.equal(a, b), f"appended buffers differ at pos {pos}"
     sta.plan.check()
@@ -87,7 +102,7 @@ def test_plans_of_other_kinds_share_the_array():
             y_sta = torch.empty_like(y_ref)
             _static_decode(sta, pos, x, y_sta)
             torch.cuda.synchronize()
-            assert torch.equal(y_sta, y_ref), (c.kind, pos)
+            assert _same_y(c.kind, y_sta, y_ref), (c.kind, pos)
     for ref, sta in pairs:
         ref.close()
         sta.close()
