@@ -112,9 +112,9 @@ def flush_bytes(cfg, rank, n: int) -> int:
 
 
 def decode_launches(cfg) -> int:
-    """Kernel launches of one sketch-decode call: the one-launch form for Mamba-2, the
-    coefficient kernel and the combine for GDN / KDA."""
-    return 1 if cfg.kind == "mamba2" else 2
+    """Kernel launches of one sketch-decode call: the products kernel (Mamba-2) or the
+    coefficient kernel (GDN / KDA), then the combine."""
+    return 2
 
 
 # ----------------------------------------------------------------------------- environment
@@ -129,16 +129,17 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s)"
 
 
-def kernel_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel's source
-    is unchanged since the counters were taken (else None)."""
+def kernel_traffic(kernel: str, workload: str = "nemotron-nano-mamba2-layer"):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary,
+    if the kernel's source is unchanged since the counters were taken (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f)[kernel]
-        src = os.path.join(ROOT, rec["source"])
-        if hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["source_sha256"]:
-            return None
+            rec = json.load(f)[f"{kernel}@{workload}"]
+        for src_rel, sha in rec["sources"].items():
+            src = os.path.join(ROOT, src_rel)
+            if hashlib.sha256(open(src, "rb").read()).hexdigest() != sha:
+                return None
         return rec
     except Exception:
         return None
@@ -260,6 +261,173 @@ def max_over_ranks(values, device=None):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+class Replicas:
+    """L independent layer replicas of one workload on one GPU (each more than 1 GB, so
+    that no launch finds its layer's data in the 126 MB L2), with W steps of inputs
+    each, and the timing loops of the hot path and its baselines.  Every loop records a
+    CUDA event pair around every launch it times, on the launching stream."""
+
+    def __init__(self, cfg, L: int, rank_id: int, dev, seed_base: int = 0):
+        import torch
+        import rank_state_read_b200 as rs
+        self.cfg, self.dev = cfg, dev
+        self.stream = torch.cuda.current_stream()
+        self.rank = synth.layer_rank_table(cfg)
+        self.omega = synth.basis(cfg)
+        self.layers, self.inputs = [], []
+        for l in range(L):
+            seed = replica_seed(rank_id, seed_base + l)
+            S0 = synth.device_state(cfg, seed, dev)
+            self.layers.append(rs.SketchLayer(cfg.kind, batch=cfg.B, heads=cfg.H, qk_heads=cfg.Hqk,
+                                              key_dim=cfg.K, value_dim=cfg.V, window=cfg.W, groups=cfg.G,
+                                              rank_cap=cfg.cap, rank=self.rank.tolist(), omega=self.omega,
+                                              S0=S0, device=dev))
+            self.inputs.append([synth.device_step_inputs(cfg, seed + 1 + p, dev) for p in range(cfg.W)])
+            del S0
+        for lay in self.layers:
+            lay.flush(0)
+        torch.cuda.synchronize()
+
+    def _ev(self):
+        import torch
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(self.stream)
+        return e
+
+    def cycle(self, dense=False, events=None):
+        """One window cycle on every replica: W decodes (the sketch decode, or the
+        dense-read decode), the last followed by the flush (sketch decode only)."""
+        cfg = self.cfg
+        for p in range(cfg.W):
+            for l, lay in enumerate(self.layers):
+                x = self.inputs[l][p]
+                e0 = self._ev() if events is not None else None
+                if dense:
+                    lay.dense_decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
+                else:
+                    lay.decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
+                if events is not None:
+                    events["decode"].append((p, e0, self._ev()))
+                if p == cfg.W - 1 and not dense:
+                    e2 = self._ev() if events is not None else None
+                    lay.flush(cfg.W)
+                    if events is not None:
+                        events["flush"].append((cfg.W, e2, self._ev()))
+
+    def dense_cycles(self, k: int):
+        """k dense-read cycles; their buffered tokens are then applied (untimed)."""
+        import torch
+        ev = {"decode": [], "flush": []}
+        for _ in range(k):
+            self.cycle(dense=True, events=ev)
+        for lay in self.layers:
+            lay.flush(self.cfg.W)
+        torch.cuda.synchronize()
+        return [(p, a, b) for p, a, b in ev["decode"]]
+
+    def standard_steps(self, k: int):
+        """k x W standard per-step decodes on every replica (same tokens)."""
+        import torch
+        out = []
+        for _ in range(k):
+            for p in range(self.cfg.W):
+                for l, lay in enumerate(self.layers):
+                    x = self.inputs[l][p]
+                    e0 = self._ev()
+                    lay.standard_step(x["q"], x["k"], x["v"], x["a"], x["beta"])
+                    out.append((e0, self._ev()))
+        torch.cuda.synchronize()
+        return out
+
+    def close(self):
+        for lay in self.layers:
+            lay.close()
+        self.layers, self.inputs = [], []
+
+
+def _mean_ms(pairs):
+    return sum(a.elapsed_time(b) for a, b in pairs) / len(pairs)
+
+
+def kernel_roof(kernel, achieved, nbytes_per_launch, peak, peak_src, workload):
+    tr = kernel_traffic(kernel, workload)
+    return {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": peak_src,
+            "algorithmic_bytes_per_launch": int(nbytes_per_launch),
+            "traffic": None if tr is None else tr["dram_bytes_per_launch_full_size"]}
+
+
+def family_record(reps: Replicas, cycles: int, peak: float, peak_src: str, barrier) -> dict:
+    """Decode, flush, dense-read decode and standard step of one workload: mean device
+    time per launch (CUDA events), algorithmic GB/s and fraction of the HBM peak, DRAM
+    traffic per launch from the committed ncu record when its source is unchanged."""
+    cfg, rank = reps.cfg, reps.rank
+    ev = {"decode": [], "flush": []}
+    barrier()
+    for _ in range(cycles):
+        reps.cycle(events=ev)
+    barrier()
+    dec = [(p, a.elapsed_time(b)) for p, a, b in ev["decode"]]
+    fl = [a.elapsed_time(b) for _, a, b in ev["flush"]]
+    dd = [(p, a.elapsed_time(b)) for p, a, b in reps.dense_cycles(max(1, cycles // 2))]
+    barrier()
+    st = reps.standard_steps(1)
+    barrier()
+    dec_us = 1e3 * sum(t for _, t in dec) / len(dec)
+    fl_us = 1e3 * sum(fl) / len(fl)
+    dd_us = 1e3 * sum(t for _, t in dd) / len(dd)
+    st_us = 1e3 * _mean_ms(st)
+    dec_b = sum(decode_bytes(cfg, rank, p) for p, _ in dec) / len(dec)
+    dd_b = sum(dense_decode_bytes(cfg, p) for p, _ in dd) / len(dd)
+    fl_b = flush_bytes(cfg, rank, cfg.W)
+    gbs = lambda nbytes, us: nbytes / (us * 1e-6) / 1e9
+    w = cfg.name
+    return {
+        "workload": w, "kind": cfg.kind, "batch": cfg.B, "heads": cfg.H, "K": cfg.K, "V": cfg.V,
+        "groups": cfg.G, "qk_heads": cfg.Hqk, "mean_rank": cfg.mean_rank,
+        "dense_heads": int((rank < 0).sum()), "layer_replicas": len(reps.layers), "window_cycles": cycles,
+        "decode": {"us": round(dec_us, 2), **kernel_roof("sketchssm_decode", gbs(dec_b, dec_us), dec_b, peak,
+                                                         peak_src, w),
+                   "launches_per_call": decode_launches(cfg)},
+        "flush": {"us": round(fl_us, 2), **kernel_roof("sketchssm_flush", gbs(fl_b, fl_us), fl_b, peak, peak_src, w)},
+        "dense_read": {"us": round(dd_us, 2), **kernel_roof("sketchssm_dense_decode", gbs(dd_b, dd_us), dd_b, peak,
+                                                             peak_src, w)},
+        "standard_step": {"us": round(st_us, 2), **kernel_roof("sketchssm_step", gbs(step_bytes(cfg), st_us),
+                                                                step_bytes(cfg), peak, peak_src, w)},
+        "window_tok_s": round(cfg.B * cfg.W / ((cfg.W * dec_us + fl_us) * 1e-6), 1),
+        "speedup_vs_dense_read": round(dd_us / dec_us, 3),
+        "traffic_ratio_dense_over_sketch": round(dd_b / dec_b, 3),
+        "speedup_vs_standard_step": round(cfg.W * st_us / (cfg.W * dec_us + fl_us), 3),
+    }
+
+
+def state_traffic(cfg, rank) -> dict:
+    """DRAM bytes per token of the sketch path (W decodes + the flush, over W tokens)
+    against the standard per-step decode, from the committed ncu record (all bytes the
+    kernels moved, the token buffers included), beside the same ratio for the state
+    alone counted from the shapes (the pages' figure is about 10x)."""
+    B, H, K, V, W = cfg.B, cfg.H, cfg.K, cfg.V, cfg.W
+    sk_rows = int(rank[rank > 0].sum())
+    nd = int((rank <= 0).sum())
+    st_state = 2 * H * K * V * 4
+    sk_state = (sk_rows * V + nd * K * V) * 4 + (2 * H * K * V + sk_rows * V) * 4 / W
+    out = {"analytic_state_bytes_per_token": {"standard_step": st_state, "sketch_path": round(sk_state, 1),
+                                              "ratio": round(st_state / sk_state, 2)},
+           "pages_ratio": "about 10x (mean sketch rank 8)"}
+    dec = kernel_traffic("sketchssm_decode", cfg.name)
+    fl = kernel_traffic("sketchssm_flush", cfg.name)
+    st = kernel_traffic("sketchssm_step", cfg.name)
+    if dec and fl and st:
+        sk = (W * dec["dram_bytes_per_launch_full_size"] + fl["dram_bytes_per_launch_full_size"]) / (W * B)
+        std = st["dram_bytes_per_launch_full_size"] / B
+        out["measured_dram_bytes_per_token"] = {"standard_step": round(std, 1), "sketch_path": round(sk, 1),
+                                                "ratio": round(std / sk, 2),
+                                                "source": "profiles/ncu_traffic.json"}
+    else:
+        out["measured_dram_bytes_per_token"] = None
+    return out
+
+
 def run_ours(args, cfg) -> None:
     import torch
     import torch.distributed as dist
@@ -273,57 +441,19 @@ def run_ours(args, cfg) -> None:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream()
-
-    rank = synth.layer_rank_table(cfg)
-    omega = synth.basis(cfg)
-    L = args.replicas
-    layers, inputs = [], []
-    for l in range(L):
-        seed = replica_seed(rank_id, l)
-        S0 = synth.device_state(cfg, seed, dev)
-        layers.append(rs.SketchLayer(cfg.kind, batch=cfg.B, heads=cfg.H, qk_heads=cfg.Hqk,
-                                     key_dim=cfg.K, value_dim=cfg.V, window=cfg.W, groups=cfg.G,
-                                     rank_cap=cfg.cap, rank=rank.tolist(), omega=omega, S0=S0,
-                                     device=dev))
-        inputs.append([synth.device_step_inputs(cfg, seed + 1 + p, dev) for p in range(cfg.W)])
-        del S0
-    for lay in layers:
-        lay.flush(0)
-    torch.cuda.synchronize()
-
-    def cycle(dense=False, events=None):
-        for p in range(cfg.W):
-            for l, lay in enumerate(layers):
-                x = inputs[l][p]
-                if events is not None:
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                if dense:
-                    lay.dense_decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
-                else:
-                    lay.decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
-                if events is not None:
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e1.record(stream)
-                    events["decode"].append((p, e0, e1))
-                if p == cfg.W - 1 and not dense:
-                    if events is not None:
-                        e2 = torch.cuda.Event(enable_timing=True)
-                        e2.record(stream)
-                    lay.flush(cfg.W)
-                    if events is not None:
-                        e3 = torch.cuda.Event(enable_timing=True)
-                        e3.record(stream)
-                        events["flush"].append((cfg.W, e2, e3))
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
+    reps = Replicas(cfg, args.replicas, rank_id, dev)
+    stream = reps.stream
+    rank, omega, layers, inputs = reps.rank, reps.omega, reps.layers, reps.inputs
+    L = len(layers)
+
     for _ in range(args.warmup):
-        cycle()
+        reps.cycle()
     barrier()
 
     # ---- timed region: K steps of the hot path
@@ -336,43 +466,24 @@ def run_ours(args, cfg) -> None:
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for _ in range(args.steps):
-        cycle(events=ev)
+        reps.cycle(events=ev)
     t_end.record(stream)
     barrier()
     clocks = sampler.stop()
     ms = t_start.elapsed_time(t_end)
     dec = [(p, a.elapsed_time(b)) for p, a, b in ev["decode"]]
     fl = [b_.elapsed_time(c_) for _, b_, c_ in ev["flush"]]
-    # a Mamba-2 sketch decode is one launch; GDN / KDA: the coefficient kernel + the combine
     launches = decode_launches(cfg) * len(ev["decode"]) + len(ev["flush"])
 
     # ---- dense-read baseline decode (same positions, same replicas)
     kd = max(1, min(args.steps, 10))
-    evd = {"decode": [], "flush": []}
     barrier()
-    for _ in range(kd):
-        cycle(dense=True, events=evd)
-    barrier()
-    dd = [(p, a.elapsed_time(b)) for p, a, b in evd["decode"]]
-    for lay in layers:   # the dense-read cycles left W tokens buffered: apply them
-        lay.flush(cfg.W)
-
+    dd = [(p, a.elapsed_time(b)) for p, a, b in reps.dense_cycles(kd)]
     # ---- standard per-step decode (full state read and updated every token), the
     # baseline the pages' speedups are quoted against: same replicas, same tokens
-    st_ev = []
     barrier()
-    for _ in range(kd):
-        for p in range(cfg.W):
-            for l, lay in enumerate(layers):
-                x = inputs[l][p]
-                e0 = torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                lay.standard_step(x["q"], x["k"], x["v"], x["a"], x["beta"])
-                e1 = torch.cuda.Event(enable_timing=True)
-                e1.record(stream)
-                st_ev.append((e0, e1))
+    st = [a.elapsed_time(b) for a, b in reps.standard_steps(kd)]
     barrier()
-    st = [a.elapsed_time(b) for a, b in st_ev]
 
     # ---- prefill handoff on replica 0: a prompt of PREFILL_T tokens applied to the state,
     # then the sketch formed (sketchssm_prefill); the kernel alone = the call with the
@@ -394,35 +505,75 @@ def run_ours(args, cfg) -> None:
             if it:  # the first round warms up
                 pf_ev[T].append((e0, e1))
     barrier()
-    pf_us = {T: 1e3 * sum(a.elapsed_time(b) for a, b in ev) / len(ev) for T, ev in pf_ev.items()}
+    pf_us = {T: 1e3 * sum(a.elapsed_time(b) for a, b in ev_) / len(ev_) for T, ev_ in pf_ev.items()}
     del prompt
 
-    # ---- end to end through the C ABI: inputs from pinned host memory, y back to host
+    # ---- end to end through the C ABI: every decode's inputs copied in from pinned host
+    # memory on one stream, its y copied out to pinned host memory on another (PCIe
+    # carries both directions at once), ordered by events; two device input slots
+    cin = torch.cuda.Stream(device=dev)
+    cout = torch.cuda.Stream(device=dev)
     host_in = [{k: (None if v is None else v.cpu().pin_memory()) for k, v in inputs[0][p].items()}
                for p in range(cfg.W)]
-    dev_in = {k: (None if v is None else torch.empty_like(v)) for k, v in inputs[0][0].items()}
+    slots = [{k: (None if v is None else torch.empty_like(v)) for k, v in inputs[0][0].items()} for _ in range(2)]
+    ready = [torch.cuda.Event() for _ in range(2)]   # a slot's inputs have landed
+    used = [torch.cuda.Event() for _ in range(2)]    # the decode that read a slot has run
+    ydone = [torch.cuda.Event() for _ in layers]     # a layer's y has been copied out
     host_y = [torch.empty(layers[0].y.shape, dtype=torch.float32).pin_memory() for _ in layers]
     ke = max(1, min(args.steps, 5))
     barrier()
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
+    cin.wait_event(e_start)
+    cout.wait_event(e_start)
     h2d = d2h = 0
+    s = 0
     for _ in range(ke):
         for p in range(cfg.W):
             for l, lay in enumerate(layers):
-                for k, v in host_in[p].items():
-                    if v is not None:
-                        dev_in[k].copy_(v, non_blocking=True)
-                        h2d += v.numel() * 4
-                y = lay.decode(p, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["a"], dev_in["beta"])
-                host_y[l].copy_(y, non_blocking=True)
+                slot = s & 1
+                cin.wait_event(used[slot])
+                with torch.cuda.stream(cin):
+                    for k, v in host_in[p].items():
+                        if v is not None:
+                            slots[slot][k].copy_(v, non_blocking=True)
+                            h2d += v.numel() * 4
+                ready[slot].record(cin)
+                stream.wait_event(ready[slot])
+                stream.wait_event(ydone[l])
+                x = slots[slot]
+                y = lay.decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
+                used[slot].record(stream)
+                cout.wait_stream(stream)
+                with torch.cuda.stream(cout):
+                    host_y[l].copy_(y, non_blocking=True)
+                ydone[l].record(cout)
                 d2h += y.numel() * 4
                 if p == cfg.W - 1:
                     lay.flush(cfg.W)
+                s += 1
+    stream.wait_stream(cin)
+    stream.wait_stream(cout)
     e_end.record(stream)
     barrier()
     e2e_ms = e_start.elapsed_time(e_end)
+    reps.close()
+    del reps, layers, inputs, slots
+
+    # ---- the other families (GDN, KDA layers) under the same clock, smaller loops
+    families = {}
+    if not args.no_families:
+        peak, peak_src = hbm_peak()
+        for cid, key in ((3, "gdn"), (4, "kda")):
+            fcfg = synth.config(cid)
+            fr = Replicas(fcfg, args.family_replicas, rank_id, dev, seed_base=200 + cid)
+            for _ in range(2):
+                fr.cycle()
+            families[key] = family_record(fr, args.family_cycles, peak, peak_src, barrier)
+            fr.close()
+            del fr
+            torch.cuda.empty_cache()
 
     # ---- max over ranks
     ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
@@ -447,16 +598,9 @@ def run_ours(args, cfg) -> None:
     mean_st_us = 1e3 * sum(st) / len(st)
     st_gbs = step_bytes(cfg) / (mean_st_us * 1e-6) / 1e9
 
-    def roof(kernel, achieved, nbytes_per_launch):
-        tr = kernel_traffic(kernel)
-        return {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": peak_src,
-                "algorithmic_bytes_per_launch": int(nbytes_per_launch),
-                "traffic": None if tr is None else tr["dram_bytes_per_launch_full_size"]}
-
     share_dec = dec_ms / (dec_ms + fl_ms)
-    r_dec = roof("sketchssm_decode", dec_gbs, dec_bytes / len(dec))
-    r_fl = roof("sketchssm_flush", fl_gbs, fl_bytes / len(fl))
+    r_dec = kernel_roof("sketchssm_decode", dec_gbs, dec_bytes / len(dec), peak, peak_src, cfg.name)
+    r_fl = kernel_roof("sketchssm_flush", fl_gbs, fl_bytes / len(fl), peak, peak_src, cfg.name)
     dominant, other = (r_dec, r_fl) if share_dec >= 0.5 else (r_fl, r_dec)
 
     line = {
@@ -476,29 +620,34 @@ def run_ours(args, cfg) -> None:
         "roofline_other": other,
         "kernel_share": {"sketchssm_decode": round(share_dec, 4), "sketchssm_flush": round(1 - share_dec, 4)},
         "decode_us": round(mean_dec_us, 2), "flush_us": round(mean_fl_us, 2),
+        "decode_launches_per_call": decode_launches(cfg),
         "decode_only_tok_s": round(cfg.B * world / (mean_dec_us / 1e6), 1),
         "dense_read": {"decode_us": round(mean_dd_us, 2), "hbm_gbs": round(dd_gbs, 1),
                        "frac": round(dd_gbs / peak, 4),
-                       "decode_only_tok_s": round(cfg.B * world / (mean_dd_us / 1e6), 1)},
+                       "decode_only_tok_s": round(cfg.B * world / (mean_dd_us / 1e6), 1),
+                       "traffic": (lambda tr: None if tr is None else tr["dram_bytes_per_launch_full_size"])(
+                           kernel_traffic("sketchssm_dense_decode", cfg.name))},
         "speedup_vs_dense_read": round(mean_dd_us / mean_dec_us, 3),
         "traffic_ratio_dense_over_sketch": round(dd_bytes / len(dd) / (dec_bytes / len(dec)), 3),
         "standard_step": {"step_us": round(mean_st_us, 2), "hbm_gbs": round(st_gbs, 1),
                           "frac": round(st_gbs / peak, 4), "tok_s": round(cfg.B / (mean_st_us * 1e-6), 1),
                           "algorithmic_bytes_per_launch": step_bytes(cfg),
                           "traffic": (lambda tr: None if tr is None else tr["dram_bytes_per_launch_full_size"])(
-                              kernel_traffic("sketchssm_step"))},
+                              kernel_traffic("sketchssm_step", cfg.name))},
         "speedup_vs_standard_step": round(cfg.W * mean_st_us / (cfg.W * mean_dec_us + mean_fl_us), 3),
-        "prefill": prefill_report(cfg, pf_us, clocks),
+        "state_traffic": state_traffic(cfg, rank),
+        "prefill": prefill_report(cfg, pf_us, clocks, peak, peak_src),
+        "configs": families,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d // ke,
                 "d2h_bytes_per_step": d2h // ke,
-                "note": "pinned host inputs copied in and y copied out around every decode call"},
+                "note": "every decode: its inputs copied in from pinned host memory (torch copies on one "
+                        "stream) before the C-ABI decode call on device pointers, y copied out to pinned "
+                        "host memory on another stream; two input slots, event-ordered"},
         "gpu_launches": launches,
         "clocks": clocks,
     }
     if rank_id == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(cfg, rank, omega)
-    for lay in layers:
-        lay.close()
     if world > 1:
         dist.destroy_process_group()
     if rank_id == 0:
@@ -507,20 +656,34 @@ def run_ours(args, cfg) -> None:
 
 # ----------------------------------------------------------------------------- reference arm
 
-def prefill_report(cfg, pf_us: dict, clocks: dict) -> dict:
-    """The prefill handoff's line: its time, prompt tok/s, and the prefill kernel's rate
-    of FP32 lane instructions against the FP32 pipe's peak (148 SMs x 128 lanes x the SM
-    clock seen under load)."""
+def prefill_bytes(cfg, T: int) -> int:
+    """Algorithmic HBM bytes of one prefill launch: the state read and written once, and
+    the prompt's T tokens (k per q/k head, v, a, beta) read, per batch row."""
+    da = cfg.K if cfg.kda else 1
+    tok = 4 * (cfg.Hqk * cfg.K + cfg.H * cfg.V + cfg.H * da + (cfg.H if cfg.has_beta else 0))
+    return cfg.B * (2 * 4 * cfg.H * cfg.K * cfg.V + T * tok)
+
+
+def prefill_report(cfg, pf_us: dict, clocks: dict, peak: float, peak_src: str) -> dict:
+    """The prefill handoff's line: its time, prompt tok/s, the prefill kernel's rate of
+    algorithmic bytes against the HBM peak (its bound once its arithmetic runs at the
+    pipe's rate), and its FP32 lane-instruction rate against the FP32 pipe's peak (148
+    SMs x 128 lanes x the SM clock seen under load), for reference."""
     T = PREFILL_T
     k_us = max(pf_us[T] - pf_us[0], 1e-3)
     mhz = clocks.get("sm_max_mhz") or 1965.0
-    peak = SMS * FP32_LANES_PER_SM * mhz * 1e6 / 1e12
+    alu_peak = SMS * FP32_LANES_PER_SM * mhz * 1e6 / 1e12
     ach = prefill_instr(cfg, T) / (k_us * 1e-6) / 1e12
+    gbs = prefill_bytes(cfg, T) / (k_us * 1e-6) / 1e9
     return {"prompt_tokens": T, "handoff_us": round(pf_us[T], 2), "sketch_only_us": round(pf_us[0], 2),
             "kernel_us": round(k_us, 2), "prompt_tok_s": round(cfg.B * T / (pf_us[T] * 1e-6), 1),
-            "roofline": {"kernel": "sketchssm_prefill", "bound": "alu", "achieved": round(ach, 2),
-                         "peak": round(peak, 2), "unit": "T FP32 lane-instr/s", "frac": round(ach / peak, 4),
-                         "algorithmic_instr_per_launch": prefill_instr(cfg, T)}}
+            "roofline": {"kernel": "sketchssm_prefill", "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(gbs / peak, 4), "peak_source": peak_src,
+                         "algorithmic_bytes_per_launch": prefill_bytes(cfg, T),
+                         "traffic": (lambda tr: None if tr is None else tr["dram_bytes_per_launch_full_size"])(
+                             kernel_traffic("sketchssm_prefill", cfg.name))},
+            "fp32_pipe": {"achieved": round(ach, 2), "peak": round(alu_peak, 2), "unit": "T FP32 lane-instr/s",
+                          "frac": round(ach / alu_peak, 4), "algorithmic_instr_per_launch": prefill_instr(cfg, T)}}
 
 
 def run_reference(args, cfg) -> None:
@@ -568,10 +731,12 @@ def run_reference(args, cfg) -> None:
 
 def run_profile_case(args, cfg) -> None:
     """A small single-layer run for a profiler (ncu -k <kernel> -s <skip> -c <count>):
-    flush(0), then `--steps` window cycles of W sketch decodes and a flush, then two
-    standard per-step decodes and a prefill handoff of 32 tokens, with no timing and no
-    JSON line.  Launch order: the initial flush, per cycle W x (products kernel, combine
-    kernel) and the flush, the two step kernels, then the prefill kernel and its flush."""
+    flush(0), then `--steps` window cycles of W sketch decodes and a flush, then W
+    dense-read decodes and a flush, then two standard per-step decodes and a prefill
+    handoff of 32 tokens, with no timing and no JSON line.  Launch order: the initial
+    flush; per cycle W sketch decodes (Mamba-2: one kernel each; GDN / KDA: the
+    coefficient kernel and the combine) and the flush; W dense-read decodes (two
+    kernels each) and the flush; the two step kernels; the prefill kernel and its flush."""
     import torch
     import rank_state_read_b200 as rs
     rank = synth.layer_rank_table(cfg)
@@ -586,6 +751,10 @@ def run_profile_case(args, cfg) -> None:
             x = xs[p]
             layer.decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
         layer.flush(cfg.W)
+    for p in range(cfg.W):  # a window of dense-read decodes
+        x = xs[p]
+        layer.dense_decode(p, x["q"], x["k"], x["v"], x["a"], x["beta"])
+    layer.flush(cfg.W)
     for p in range(2):  # then two standard per-step decodes (step_kernel)
         x = xs[p]
         layer.standard_step(x["q"], x["k"], x["v"], x["a"], x["beta"])
@@ -607,6 +776,9 @@ def main():
     ap.add_argument("--replicas", type=int, default=8)
     ap.add_argument("--ref-rows", type=int, default=32)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-families", action="store_true", help="skip the GDN / KDA sub-records")
+    ap.add_argument("--family-replicas", type=int, default=4)
+    ap.add_argument("--family-cycles", type=int, default=6)
     ap.add_argument("--profile", action="store_true",
                     help="small single-layer run for a profiler: no timing, no JSON line")
     args = ap.parse_args()

@@ -344,12 +344,13 @@ combine_kernel(const DecodeArgs A)
         rec_list = A.rec + (size_t)(n - 1) * (H + A.G) * 8;
     }
     // the item's record: {entry, span, member mask, rows R, off[h_first], coff[h_first], coef floats, h_first}
-    int R, yrow0, c0, cfl, h_first;
+    int R, yrow0, c0, cfl, h_first, span;
     unsigned mask;
     bool dense;
     if (A.dense_all) {
         dense = true;
         h_first = blockIdx.x;
+        span = 1;
         mask = 1u;
         R = KDIM;
         yrow0 = 0;
@@ -359,6 +360,7 @@ combine_kernel(const DecodeArgs A)
         const int4 r0 = __ldg(reinterpret_cast<const int4 *>(rec_list) + 2 * blockIdx.x);
         const int4 r1 = __ldg(reinterpret_cast<const int4 *>(rec_list) + 2 * blockIdx.x + 1);
         dense = r0.x < 0;
+        span = r0.y;
         mask = (unsigned)r0.z;
         R = r0.w;
         yrow0 = r1.x;
@@ -392,12 +394,18 @@ combine_kernel(const DecodeArgs A)
             if (M2 && dense) bulk_copy_g2s(qrow_s, A.q + ((long long)b * A.Hqk + qk) * KDIM, KDIM * 4, bar);
         }
         __syncwarp();
+        // stage rows: [item's Y block or state: R][member slot's buffered values: pos each]
+        // [the step's values: one per member]; when the members are a contiguous run of
+        // heads their step values are one contiguous run of v, so one copy brings them all
         const long long bh = (long long)b * H + h;
         if (member) {
-            float *dst = stage + (size_t)(R + slot * n) * V;
-            if (pos > 0) bulk_copy_g2s(dst, A.vbuf + bh * W * V, (uint32_t)(pos * V * 4), bar);
-            bulk_copy_g2s(dst + (size_t)pos * V, A.v + bh * V, (uint32_t)(V * 4), bar);
+            if (pos > 0)
+                bulk_copy_g2s(stage + (size_t)(R + slot * pos) * V, A.vbuf + bh * W * V, (uint32_t)(pos * V * 4), bar);
+            if (span != nh) bulk_copy_g2s(stage + (size_t)(R + nh * pos + slot) * V, A.v + bh * V, (uint32_t)(V * 4), bar);
         }
+        if (span == nh && lane == 0)
+            bulk_copy_g2s(stage + (size_t)(R + nh * pos) * V, A.v + ((long long)b * H + h_first) * V,
+                          (uint32_t)(nh * V * 4), bar);
         // the products of the first launch of this step: wait until it has finished
         pdl_wait_primary();
         if (!M2 && lane == 0)
@@ -453,16 +461,19 @@ combine_kernel(const DecodeArgs A)
     const int V4 = V >> 2;
     for (int o = tid; o < nh * V4; o += blockDim.x) {
         const int hl = o / V4, c4 = o - hl * V4;
-        const int r0 = rbs[hl], rbh = rb[hl], rr = R + hl * n;
+        const int r0 = rbs[hl], rbh = rb[hl];
+        const int rv = R + hl * pos, rcur = R + nh * pos + hl;  // buffered values, the step's value
         const float *sp = stage + c4 * 4;
         float4 acc0 = zero4(), acc1 = zero4();
         if (M2) {
             const float *sv = dots + (size_t)ch[hl] * dr;
             const float *uv = dense ? qrow_s : sv + W;
             const float *av = as_s + hl * W;
-            float w = 1.f;  // prod_{j>i} a_j, newest token first; ends as decay_prod
-            for (int i = n - 1; i >= 0; --i) {
-                fma4(acc1, w * sv[i], lds4(sp + (size_t)(rr + i) * V));
+            // prod_{j>i} a_j, newest token first; ends as decay_prod
+            fma4(acc1, sv[pos], lds4(sp + (size_t)rcur * V));
+            float w = av[pos];
+            for (int i = pos - 1; i >= 0; --i) {
+                fma4(acc1, w * sv[i], lds4(sp + (size_t)(rv + i) * V));
                 w *= av[i];
             }
             int j = 0;
@@ -479,12 +490,13 @@ combine_kernel(const DecodeArgs A)
                 fma4(acc1, cf[j + 1], lds4(sp + (size_t)(r0 + j + 1) * V));
             }
             if (j < rbh) fma4(acc0, cf[j], lds4(sp + (size_t)(r0 + j) * V));
-            for (int i = 0; i < n; ++i) fma4(acc1, cf[rbh + i], lds4(sp + (size_t)(rr + i) * V));
+            for (int i = 0; i < pos; ++i) fma4(acc1, cf[rbh + i], lds4(sp + (size_t)(rv + i) * V));
+            fma4(acc1, cf[rbh + pos], lds4(sp + (size_t)rcur * V));
         }
         const float4 acc = make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
         const long long bh = (long long)b * H + hs[hl];
         st4(A.y + bh * V + c4 * 4, acc);
-        st4(A.vbuf + (bh * W + pos) * V + c4 * 4, lds4(sp + (size_t)(rr + pos) * V));
+        st4(A.vbuf + (bh * W + pos) * V + c4 * 4, lds4(sp + (size_t)rcur * V));
     }
 }
 

@@ -86,7 +86,7 @@ __host__ __device__ inline FlushCarve flush_carve(int kind, int VS, int W, int r
     o = align128(o + 2 * sizeof(float) * c.tfloats);
     c.O = o;
     o = align128(o + sizeof(float) * (size_t)rcap * KDIM);
-    c.AF = o;  // Mamba-2: split key fragments, [k-step][m-tile][lane][hi 4, lo 4]
+    c.AF = o;  // Mamba-2: split key fragments, [k-step][m-tile][hi, lo][lane][4]
     o = align128(o + (m2 ? sizeof(float) * (size_t)((W + 7) / 8) * 8 * 32 * 8 : 0));
     c.total = o;
     return c;
@@ -470,7 +470,9 @@ flush_kernel(const FlushArgs A)
                         for (int e = 0; e < 4; ++e) c[mt][nt][e] *= P;
                 // the keys' A fragments, split hi / lo once per key set (shared by the
                 // heads of a q/k head): all compute warps build them between two named
-                // barriers; tokens >= n are 0
+                // barriers; tokens >= n are 0.  Stored [k-step][m-tile][hi | lo][lane][4], so
+                // that the 128-bit fragment reads of a warp are 512 consecutive bytes (no
+                // bank conflict)
                 const long long key = (long long)cur.b * A.Hqk + cur.h / A.hpq;
                 if (key != af_key) {
                     af_key = key;
@@ -483,9 +485,9 @@ flush_kernel(const FlushArgs A)
                         const float v = (ok && tok < n) ? kt[(size_t)tok * cv.ks + srow(mt, ln >> 2, comp & 1)] : 0.f;
                         uint32_t hi, lo;
                         split_tf32(v, hi, lo);
-                        float *f = AF + (size_t)((k8 * 8 + mt) * 32 + ln) * 8;
+                        float *f = AF + (size_t)((k8 * 8 + mt) * 64 + ln) * 4;  // lo 128 floats on
                         f[comp] = __uint_as_float(hi);
-                        f[4 + comp] = __uint_as_float(lo);
+                        f[128 + comp] = __uint_as_float(lo);
                     }
                     compute_barrier(ncw);
                 }
@@ -504,11 +506,11 @@ flush_kernel(const FlushArgs A)
                         split_tf32(v0, bh[nt][0], bl[nt][0]);
                         split_tf32(v1, bh[nt][1], bl[nt][1]);
                     }
-                    const float *af = AF + (size_t)((k0 >> 3) * 8 * 32 + lane) * 8;
+                    const float *af = AF + (size_t)((k0 >> 3) * 8 * 64 + lane) * 4;
 #pragma unroll
                     for (int mt = 0; mt < 8; ++mt) {
-                        const uint4 fh = *reinterpret_cast<const uint4 *>(af + mt * 32 * 8);
-                        const uint4 fl = *reinterpret_cast<const uint4 *>(af + mt * 32 * 8 + 4);
+                        const uint4 fh = *reinterpret_cast<const uint4 *>(af + mt * 64 * 4);
+                        const uint4 fl = *reinterpret_cast<const uint4 *>(af + mt * 64 * 4 + 128);
                         const uint32_t ah[4] = {fh.x, fh.y, fh.z, fh.w}, al[4] = {fl.x, fl.y, fl.z, fl.w};
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt) {

@@ -85,11 +85,6 @@ int dots_row(int W, int cap);
 size_t decode_smem_bytes(const DecodeArgs &a);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
-// Mamba-2 sketch decode in one launch, one CTA per (basis group, batch row), no scratch:
-// used when the layer's shape fits (Mamba-2, not the dense-read baseline).
-bool decode_group_supported(const DecodeArgs &a);
-size_t decode_group_smem(const DecodeArgs &a);
-cudaError_t launch_decode_group(const DecodeArgs &a, cudaStream_t stream);
 
 // Arguments of one standard per-step decode launch.
 struct StepArgs {

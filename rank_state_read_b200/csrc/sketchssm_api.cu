@@ -519,8 +519,7 @@ sketchssm_status sketchssm_decode_rows(const sketchssm_plan *p, const int32_t *p
     int most = 0;
     for (int c : p->h_items) most = c > most ? c : most;
     A.n_items = most;
-    cudaError_t e = sk::decode_group_supported(A) ? sk::launch_decode_group(A, (cudaStream_t)stream)
-                                                  : sk::launch_decode(A, (cudaStream_t)stream);
+    cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     return SKETCHSSM_OK;
 }
@@ -541,8 +540,7 @@ sketchssm_status sketchssm_decode(const sketchssm_plan *p, int32_t pos, const fl
     CHECK_T(omega, any_sketch ? fbytes(d.groups, d.basis_rows, d.key_dim) : 0, "omega", !any_sketch);
     CHECK_T(S, any_dense ? fbytes(d.batch, d.heads, d.key_dim, d.value_dim) : 0, "S", !any_dense);
     const sk::DecodeArgs A = decode_args(p, pos, q, k, v, a, beta, kbuf, vbuf, abuf, bbuf, Y, omega, S, y, 0);
-    cudaError_t e = sk::decode_group_supported(A) ? sk::launch_decode_group(A, (cudaStream_t)stream)
-                                                  : sk::launch_decode(A, (cudaStream_t)stream);
+    cudaError_t e = sk::launch_decode(A, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     return SKETCHSSM_OK;
 }

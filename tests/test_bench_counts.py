@@ -50,3 +50,22 @@ def test_prefill_instruction_counts():
     for cid, per in ((1, 1), (3, 2), (4, 3)):
         cfg = synth.config(cid)
         assert bench.prefill_instr(cfg, 64) == per * cfg.B * cfg.H * cfg.K * cfg.V * 64
+
+
+def test_prefill_bytes_of_the_mamba2_layer():
+    """The prefill reads and writes the state once and reads every prompt token:
+    2 x 256 x 128 x 128 x 80 x 4 bytes + 64 tokens x 256 rows x (8 x 128 + 128 x 80 + 128) x 4."""
+    cfg = synth.config(1)
+    state = 2 * 256 * 128 * 128 * 80 * 4
+    toks = 64 * 256 * 4 * (8 * 128 + 128 * 80 + 128)
+    assert bench.prefill_bytes(cfg, 64) == state + toks
+
+
+def test_state_traffic_ratio_of_the_shapes():
+    """The state-only bytes per token of the standard step over those of the sketch path
+    (SURVEY's reconstruction of the pages' figure: 10.4x at rank 8, W = 16, K = 128,
+    V = 80, no dense head)."""
+    cfg = synth.config(1).replace(n_dense=0)
+    rank = np.full(cfg.H, 8, np.int32)
+    r = bench.state_traffic(cfg, rank)["analytic_state_bytes_per_token"]
+    assert abs(r["ratio"] - 10.4) < 0.05
