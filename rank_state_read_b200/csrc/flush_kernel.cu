@@ -263,7 +263,7 @@ __device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
 // d = D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1])
 __device__ __forceinline__ void mma_tf32(float *d, const uint32_t *a, const uint32_t *b)
 {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

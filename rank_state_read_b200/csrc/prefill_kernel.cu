@@ -5,13 +5,19 @@
 // M = a I, beta = 1; GDN: M = a (I - beta k k^T); KDA: M = diag(a) (I - beta k k^T)).
 // The host then forms the sketch with the n = 0 flush.
 //
-// One CTA per (b, h, column slab of VS columns), 2 VS threads.  The slab stays in
-// registers for the whole prompt (thread (ks, c4) holds the float4 column chunk c4 of
-// the 16 state rows 4 ks + 32 q + e, q, e < 4), so S is read and written once however
-// long the prompt; the delta rule's k^T S is 3 xor-shuffle steps inside the warp.  The
-// prompt comes through shared memory in chunks of PF_CHUNK tokens, double buffered with
-// cp.async: chunk c + 1 is in flight while the CTA applies chunk c.  No thread waits
-// on another CTA or on a flag: the only waits are cp.async groups and CTA barriers.
+// One CTA per (b, h, column slab of VS columns), 2 VS threads, the slab held in
+// registers for the whole prompt, so S is read and written once however long the
+// prompt.  The prompt comes through shared memory in chunks of PF_CHUNK tokens, double
+// buffered with cp.async: chunk c + 1 is in flight while the CTA applies chunk c.  No
+// thread waits on another CTA or on a flag: the only waits are cp.async groups and CTA
+// barriers.
+//   Mamba-2 (prefill_tc_kernel): a chunk of n tokens is one contraction,
+//     S <- P S + K^T (w o V), w_i = product of the later decays in the chunk, P of all,
+//     on the tensor cores (mma.sync m16n8k8, tf32 operands split hi + lo, three
+//     products, fp32 accumulators holding the state in the flush's layout).
+//   GDN / KDA (prefill_kernel): thread (ks, c4) holds the float4 column chunk c4 of the
+//     16 state rows 4 ks + 32 q + e, and applies the delta rule token by token; k^T S
+//     is 3 xor-shuffle steps inside the warp.
 #include "device_util.cuh"
 #include "internal.cuh"
 #include "ptx_util.cuh"
@@ -195,6 +201,192 @@ __global__ void __launch_bounds__(PF_MAXT) prefill_kernel(const PrefillArgs A)
         for (int e = 0; e < 4; ++e) st4(Sg + (long long)(32 * q + e) * V, s[4 * q + e]);
 }
 
+// ---------------------------------------------------------------- Mamba-2 on the tensor cores
+// Over a chunk of n <= 16 tokens the state update is S <- P S + K^T (w o V) (w_i = product
+// of the later decays in the chunk, P of all of them): a contraction with inner dimension
+// n.  It runs as mma.sync m16n8k8 with tf32 operands split x = hi + lo and the three
+// products hi hi + hi lo + lo hi accumulated in fp32, the state held in the accumulators
+// for the whole prompt.  Warp w owns columns 16 w .. 16 w + 15 of the slab for all 128
+// rows: c[mt][nt][2 h + e] = state row srow(mt, g, h), column 16 w + 8 nt + 2 t + e
+// (lane 4 g + t).
+
+__device__ __forceinline__ void pf_split_tf32(float x, uint32_t &hi, uint32_t &lo)
+{
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+    const float rest = x - __uint_as_float(hi);
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(rest));
+}
+
+__device__ __forceinline__ void pf_mma_tf32(float *d, const uint32_t *a, const uint32_t *b)
+{
+    asm(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// accumulator row 16 mt + g + 8 h <-> state row (a bijection of 0 .. 127)
+__device__ __forceinline__ int pf_srow(int mt, int g, int h) { return 8 * g + 4 * h + 64 * (mt >> 2) + (mt & 3); }
+
+struct TcCarve {
+    size_t k, v, a, af, total;
+    int vsp;  // padded value row: the B-fragment reads of a warp fall on 32 banks
+};
+
+__host__ __device__ inline TcCarve tc_carve(int VS)
+{
+    TcCarve c;
+    c.vsp = VS + 8;
+    size_t o = 0;
+    c.k = o;
+    o = pf_align(o + sizeof(float) * 2 * PF_CHUNK * KDIM);
+    c.v = o;
+    o = pf_align(o + sizeof(float) * 2 * PF_CHUNK * (size_t)c.vsp);
+    c.a = o;  // decays [2][PF_CHUNK], then the chunk's w_i [PF_CHUNK] and P
+    o = pf_align(o + sizeof(float) * (3 * PF_CHUNK + 1));
+    c.af = o;  // [k-step][m-tile][hi, lo][lane][4]
+    o = pf_align(o + sizeof(float) * (PF_CHUNK / 8) * 8 * 32 * 8);
+    c.total = o;
+    return c;
+}
+
+__global__ void __launch_bounds__(PF_MAXT, 3) prefill_tc_kernel(const PrefillArgs A)
+{
+    extern __shared__ __align__(128) unsigned char psm[];
+    const int V = A.V, VS = A.VS, nslab = V / VS, T = A.T;
+    const TcCarve cv = tc_carve(VS);
+    float *ks_ = reinterpret_cast<float *>(psm + cv.k);
+    float *vs_ = reinterpret_cast<float *>(psm + cv.v);
+    float *as_ = reinterpret_cast<float *>(psm + cv.a);
+    float *AF = reinterpret_cast<float *>(psm + cv.af);
+    const int vsp = cv.vsp;
+
+    const long long item = blockIdx.x;
+    const long long bh = item / nslab;
+    const int slab = (int)(item - bh * nslab);
+    const long long b = bh / A.H;
+    const int h = (int)(bh - b * A.H), qk = h / A.hpq;
+    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t = lane & 3, col0 = warp * 16;
+    const int nchunk = (T + PF_CHUNK - 1) / PF_CHUNK;
+
+    // copies of tokens t0 .. t0 + n - 1 into stage st
+    auto issue = [&](int t0, int n, int st) {
+        const long long tb = b * A.T + t0;
+        float *kd = ks_ + st * PF_CHUNK * KDIM, *vd = vs_ + st * PF_CHUNK * vsp, *ad = as_ + st * PF_CHUNK;
+        for (int x = tid; x < n * (KDIM / 4); x += nthr) {
+            const int i = x >> 5, c = x & 31;
+            cp_async16(kd + i * KDIM + c * 4, A.k + ((tb + i) * A.Hqk + qk) * KDIM + c * 4);
+        }
+        const int vq = VS / 4;
+        for (int x = tid; x < n * vq; x += nthr) {
+            const int i = x / vq, c = x - i * vq;
+            cp_async16(vd + i * vsp + c * 4, A.v + ((tb + i) * A.H + h) * A.V + (long long)slab * VS + c * 4);
+        }
+        if (tid < n) cp_async4(ad + tid, A.a + (tb + tid) * A.H + h);
+    };
+    issue(0, min(PF_CHUNK, T), 0);
+    cp_async_commit();
+
+    float *Sg = A.S + bh * KDIM * V + (long long)slab * VS + col0 + 2 * t;
+    float c[8][2][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float2 lo = *reinterpret_cast<const float2 *>(Sg + (long long)pf_srow(mt, g, 0) * V + 8 * nt);
+            const float2 hi = *reinterpret_cast<const float2 *>(Sg + (long long)pf_srow(mt, g, 1) * V + 8 * nt);
+            c[mt][nt][0] = lo.x;
+            c[mt][nt][1] = lo.y;
+            c[mt][nt][2] = hi.x;
+            c[mt][nt][3] = hi.y;
+        }
+
+    for (int ch = 0; ch < nchunk; ++ch) {
+        const int st = ch & 1;
+        cp_async_wait<0>();
+        __syncthreads();  // chunk ch has landed; every warp is done with chunk ch - 1
+        if (ch + 1 < nchunk) {
+            const int t1 = (ch + 1) * PF_CHUNK;
+            issue(t1, min(PF_CHUNK, T - t1), st ^ 1);
+        }
+        cp_async_commit();
+        const int n = min(PF_CHUNK, T - ch * PF_CHUNK);
+        const float *kt = ks_ + st * PF_CHUNK * KDIM;
+        const float *vt = vs_ + st * PF_CHUNK * vsp + col0 + g;
+        const float *at = as_ + st * PF_CHUNK;
+        // the keys' A fragments of this chunk, split hi / lo; tokens >= n are 0
+        const int nkt = (n + 7) >> 3;
+        for (int x = tid; x < nkt * 8 * 32 * 4; x += nthr) {
+            const int comp = x & 3, ln = (x >> 2) & 31, mt = (x >> 7) & 7, k8 = x >> 10;
+            const int tok = 8 * k8 + (ln & 3) + 4 * (comp >> 1);
+            const float v = tok < n ? kt[tok * KDIM + pf_srow(mt, ln >> 2, comp & 1)] : 0.f;
+            uint32_t hi, lo;
+            pf_split_tf32(v, hi, lo);
+            float *f = AF + ((k8 * 8 + mt) * 64 + ln) * 4;  // hi, then lo 128 floats on
+            f[comp] = __uint_as_float(hi);
+            f[128 + comp] = __uint_as_float(lo);
+        }
+        // w_i = product of the decays after token i in the chunk (0 past the chunk), P of all
+        float *wc = as_ + 2 * PF_CHUNK;
+        if (warp == 0) {
+            float x = lane < n ? at[lane] : 1.f;  // suffix products over the lanes
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, x, o);
+                if (lane + o < 32) x *= y;
+            }
+            const float wl = __shfl_down_sync(0xffffffffu, x, 1);
+            if (lane < PF_CHUNK) wc[lane] = lane < n ? (lane == 31 ? 1.f : wl) : 0.f;
+            if (lane == 0) wc[PF_CHUNK] = x;
+        }
+        __syncthreads();  // the fragments and the weights are complete
+        const float P = wc[PF_CHUNK];
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) c[mt][nt][e] *= P;
+        for (int k0 = 0; k0 < n; k0 += 8) {
+            const int i0 = k0 + t, i1 = k0 + t + 4;
+            const float w0 = wc[i0], w1 = wc[i1];  // products of the decays after token i0, i1
+            uint32_t bhf[2][2], blf[2][2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const float v0 = i0 < n ? w0 * vt[i0 * vsp + 8 * nt] : 0.f;
+                const float v1 = i1 < n ? w1 * vt[i1 * vsp + 8 * nt] : 0.f;
+                pf_split_tf32(v0, bhf[nt][0], blf[nt][0]);
+                pf_split_tf32(v1, bhf[nt][1], blf[nt][1]);
+            }
+            const float *af = AF + ((k0 >> 3) * 8 * 64 + lane) * 4;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                const uint4 fh = *reinterpret_cast<const uint4 *>(af + mt * 64 * 4);
+                const uint4 fl = *reinterpret_cast<const uint4 *>(af + mt * 64 * 4 + 128);
+                const uint32_t ah[4] = {fh.x, fh.y, fh.z, fh.w}, al[4] = {fl.x, fl.y, fl.z, fl.w};
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    pf_mma_tf32(c[mt][nt], al, bhf[nt]);
+                    pf_mma_tf32(c[mt][nt], ah, blf[nt]);
+                    pf_mma_tf32(c[mt][nt], ah, bhf[nt]);
+                }
+            }
+        }
+    }
+
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            *reinterpret_cast<float2 *>(Sg + (long long)pf_srow(mt, g, 0) * V + 8 * nt) =
+                make_float2(c[mt][nt][0], c[mt][nt][1]);
+            *reinterpret_cast<float2 *>(Sg + (long long)pf_srow(mt, g, 1) * V + 8 * nt) =
+                make_float2(c[mt][nt][2], c[mt][nt][3]);
+        }
+}
+
 template <int KIND>
 cudaError_t launch_kind(const PrefillArgs &a, cudaStream_t stream)
 {
@@ -212,7 +404,14 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream)
 {
     if (a.B == 0 || a.T == 0) return cudaSuccess;
     switch (a.kind) {
-    case SKETCHSSM_MAMBA2: return launch_kind<SKETCHSSM_MAMBA2>(a, stream);
+    case SKETCHSSM_MAMBA2: {
+        const size_t smem = tc_carve(a.VS).total;
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const long long items = (long long)a.B * a.H * (a.V / a.VS);
+        prefill_tc_kernel<<<(unsigned)items, 2 * a.VS, smem, stream>>>(a);
+        return cudaGetLastError();
+    }
     case SKETCHSSM_GDN: return launch_kind<SKETCHSSM_GDN>(a, stream);
     default: return launch_kind<SKETCHSSM_KDA>(a, stream);
     }
