@@ -398,6 +398,7 @@ def family_record(reps: Replicas, cycles: int, peak: float, peak_src: str, barri
         "speedup_vs_dense_read": round(dd_us / dec_us, 3),
         "traffic_ratio_dense_over_sketch": round(dd_b / dec_b, 3),
         "speedup_vs_standard_step": round(cfg.W * st_us / (cfg.W * dec_us + fl_us), 3),
+        "state_traffic": state_traffic(cfg, rank),
     }
 
 

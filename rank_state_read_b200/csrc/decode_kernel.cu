@@ -67,7 +67,8 @@ __device__ __forceinline__ int row_position(const DecodeArgs &A, int b)
 // ============================================================================ query-side products
 
 constexpr int CM_THREADS = 256;
-constexpr int CM_MAXROWS = 4;
+constexpr int CM_MINROWS = 4;   // batch rows per products CTA, at least
+constexpr int CM_MAXROWS = 16;  // and at most
 constexpr int OPAD = KDIM + 4;  // padded row: threads reading different rows hit different banks
 
 struct CmCarve {
@@ -552,11 +553,20 @@ bool decode_geometry(int kind, int V, int W, int cap, int Hg, DecodeGeometry *gm
 
 int coef_block(int rows, int W) { return round4(rows + W); }
 
-int coef_rows(int cap, int W)
+int coef_rows(int cap, int W, int B, int Hqk, int sms)
 {
-    (void)cap;
-    (void)W;
-    return CM_MAXROWS;  // batch rows per Mamba-2 product CTA
+    // the fewest batch rows per CTA (at least CM_MINROWS) whose grid of Hqk x B / rows
+    // CTAs runs in one wave at the occupancy its shared memory allows: a partial second
+    // wave would cost a whole CTA lifetime of this latency-bound kernel
+    for (int rows = CM_MINROWS; rows <= CM_MAXROWS; ++rows) {
+        const size_t smem = cm_carve(cap, W, rows).total;
+        int per_sm = (int)((227 * 1024) / (smem + 1024));
+        if (per_sm > 2048 / CM_THREADS) per_sm = 2048 / CM_THREADS;
+        if (per_sm < 1) break;
+        const long long ctas = (long long)Hqk * ((B + rows - 1) / rows);
+        if (ctas <= (long long)sms * per_sm) return rows;
+    }
+    return CM_MINROWS;
 }
 
 size_t decode_smem_bytes(const DecodeArgs &a)

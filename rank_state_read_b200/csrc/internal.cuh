@@ -80,7 +80,7 @@ struct DecodeGeometry {
 };
 bool decode_geometry(int kind, int V, int W, int cap, int Hg, DecodeGeometry *gm);
 int coef_block(int rows, int W);  // floats of one head's coefficient block
-int coef_rows(int cap, int W);
+int coef_rows(int cap, int W, int B, int Hqk, int sms);  // batch rows per Mamba-2 products CTA
 int dots_row(int W, int cap);
 size_t decode_smem_bytes(const DecodeArgs &a);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
@@ -129,6 +129,7 @@ struct sketchssm_plan {
     int n_dense;
     sk::DecodeGeometry geo;
     int device;
+    int sms;  // SMs of the plan's device
     long long wait_limit;
     int coef_row;
     int *d_rank, *d_off, *d_rmax, *d_coff, *d_work, *d_rec, *d_qk_rneed, *d_counts, *d_status;

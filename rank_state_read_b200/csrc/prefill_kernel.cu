@@ -232,15 +232,17 @@ __device__ __forceinline__ int pf_srow(int mt, int g, int h) { return 8 * g + 4 
 struct TcCarve {
     size_t k, v, a, af, total;
     int vsp;  // padded value row: the B-fragment reads of a warp fall on 32 banks
+    int ksp;  // padded key row: the fragment-building reads spread over 8 bank groups, not 4
 };
 
 __host__ __device__ inline TcCarve tc_carve(int VS)
 {
     TcCarve c;
     c.vsp = VS + 8;
+    c.ksp = KDIM + 4;
     size_t o = 0;
     c.k = o;
-    o = pf_align(o + sizeof(float) * 2 * PF_CHUNK * KDIM);
+    o = pf_align(o + sizeof(float) * 2 * PF_CHUNK * (size_t)c.ksp);
     c.v = o;
     o = pf_align(o + sizeof(float) * 2 * PF_CHUNK * (size_t)c.vsp);
     c.a = o;  // decays [2][PF_CHUNK], then the chunk's w_i [PF_CHUNK] and P
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(PF_MAXT, 3) prefill_tc_kernel(const PrefillArg
     float *vs_ = reinterpret_cast<float *>(psm + cv.v);
     float *as_ = reinterpret_cast<float *>(psm + cv.a);
     float *AF = reinterpret_cast<float *>(psm + cv.af);
-    const int vsp = cv.vsp;
+    const int vsp = cv.vsp, ksp = cv.ksp;
 
     const long long item = blockIdx.x;
     const long long bh = item / nslab;
@@ -274,10 +276,10 @@ __global__ void __launch_bounds__(PF_MAXT, 3) prefill_tc_kernel(const PrefillArg
     // copies of tokens t0 .. t0 + n - 1 into stage st
     auto issue = [&](int t0, int n, int st) {
         const long long tb = b * A.T + t0;
-        float *kd = ks_ + st * PF_CHUNK * KDIM, *vd = vs_ + st * PF_CHUNK * vsp, *ad = as_ + st * PF_CHUNK;
+        float *kd = ks_ + st * PF_CHUNK * ksp, *vd = vs_ + st * PF_CHUNK * vsp, *ad = as_ + st * PF_CHUNK;
         for (int x = tid; x < n * (KDIM / 4); x += nthr) {
             const int i = x >> 5, c = x & 31;
-            cp_async16(kd + i * KDIM + c * 4, A.k + ((tb + i) * A.Hqk + qk) * KDIM + c * 4);
+            cp_async16(kd + i * ksp + c * 4, A.k + ((tb + i) * A.Hqk + qk) * KDIM + c * 4);
         }
         const int vq = VS / 4;
         for (int x = tid; x < n * vq; x += nthr) {
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(PF_MAXT, 3) prefill_tc_kernel(const PrefillArg
         }
         cp_async_commit();
         const int n = min(PF_CHUNK, T - ch * PF_CHUNK);
-        const float *kt = ks_ + st * PF_CHUNK * KDIM;
+        const float *kt = ks_ + st * PF_CHUNK * ksp;
         const float *vt = vs_ + st * PF_CHUNK * vsp + col0 + g;
         const float *at = as_ + st * PF_CHUNK;
         // the keys' A fragments of this chunk, split hi / lo; tokens >= n are 0
@@ -321,7 +323,7 @@ __global__ void __launch_bounds__(PF_MAXT, 3) prefill_tc_kernel(const PrefillArg
         for (int x = tid; x < nkt * 8 * 32 * 4; x += nthr) {
             const int comp = x & 3, ln = (x >> 2) & 31, mt = (x >> 7) & 7, k8 = x >> 10;
             const int tok = 8 * k8 + (ln & 3) + 4 * (comp >> 1);
-            const float v = tok < n ? kt[tok * KDIM + pf_srow(mt, ln >> 2, comp & 1)] : 0.f;
+            const float v = tok < n ? kt[tok * ksp + pf_srow(mt, ln >> 2, comp & 1)] : 0.f;
             uint32_t hi, lo;
             pf_split_tf32(v, hi, lo);
             float *f = AF + ((k8 * 8 + mt) * 64 + ln) * 4;  // hi, then lo 128 floats on

@@ -160,7 +160,7 @@ sk::DecodeArgs decode_args(const sketchssm_plan *p, int pos, const float *q, con
     A.dense_all = dense_all;
     A.threads = p->geo.threads;
     A.stage_rows = p->geo.stage_rows;
-    A.cm_rows = sk::coef_rows(d.rank_cap, d.window);
+    A.cm_rows = sk::coef_rows(d.rank_cap, d.window, d.batch, d.qk_heads, p->sms);
     A.dots_row = sk::dots_row(d.window, d.rank_cap);
     A.maxnh = p->geo.maxnh;
     A.coef_cap = p->geo.coef_cap;
@@ -275,6 +275,8 @@ sketchssm_status sketchssm_plan_create(const sketchssm_desc *desc, const int32_t
         return fail(SKETCHSSM_ERR_UNSUPPORTED, "a decode work item of this shape does not fit in shared memory");
     }
     cudaGetDevice(&p->device);
+    p->sms = 148;
+    cudaDeviceGetAttribute(&p->sms, cudaDevAttrMultiProcessorCount, p->device);
     p->d_rank = p->d_off = p->d_rmax = p->d_coff = p->d_work = p->d_rec = p->d_qk_rneed = nullptr;
     p->d_counts = p->d_status = nullptr;
     p->d_scratch = nullptr;
