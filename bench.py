@@ -665,26 +665,62 @@ def prefill_bytes(cfg, T: int) -> int:
     return cfg.B * (2 * 4 * cfg.H * cfg.K * cfg.V + T * tok)
 
 
+def prefill_tensor_path(cfg, T: int) -> bool:
+    """Whether the library applies this prompt on the tensor cores (the tcgen05 kernel:
+    Mamba-2, at most 64 tokens, V a multiple of 16 up to 128)."""
+    return cfg.kind == "mamba2" and 1 <= T <= 64 and cfg.V % 16 == 0 and cfg.V <= 128
+
+
+def prefill_flops(cfg, T: int) -> dict:
+    """Tensor-core work of one Mamba-2 prefill launch: the contraction's algorithmic
+    FLOPs, 2 K V T per head, and the FLOPs the kernel issues, three tf32 products (hi/lo
+    split) of M = 128 value rows (V padded) x N = K state rows x the prompt padded to 8."""
+    heads = cfg.B * cfg.H
+    tp = (T + 7) // 8 * 8
+    return {"algorithmic": 2 * heads * cfg.K * cfg.V * T, "issued": 3 * 2 * heads * 128 * cfg.K * tp}
+
+
+def tf32_peak():
+    """Dense tf32 tensor peak: the measured bf16 burst figure x the nominal tf32/bf16
+    ratio (1.1 / 2.25 PFLOP/s)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]) * 1.1 / 2.25, "measured bf16 burst x nominal tf32/bf16 ratio"
+    except Exception:
+        return 1590.0 * 1.1 / 2.25, "fallback bf16 (1.59 PFLOP/s) x nominal tf32/bf16 ratio"
+
+
 def prefill_report(cfg, pf_us: dict, clocks: dict, peak: float, peak_src: str) -> dict:
     """The prefill handoff's line: its time, prompt tok/s, the prefill kernel's rate of
-    algorithmic bytes against the HBM peak (its bound once its arithmetic runs at the
-    pipe's rate), and its FP32 lane-instruction rate against the FP32 pipe's peak (148
-    SMs x 128 lanes x the SM clock seen under load), for reference."""
+    algorithmic bytes against the HBM peak (its bound once its arithmetic keeps up), and
+    the rate of its arithmetic: for the tensor-core (Mamba-2) kernel its FLOP rate
+    against the tf32 tensor peak; otherwise its FP32 lane-instruction rate against the
+    FP32 pipe's peak (148 SMs x 128 lanes x the SM clock)."""
     T = PREFILL_T
     k_us = max(pf_us[T] - pf_us[0], 1e-3)
-    mhz = clocks.get("sm_max_mhz") or 1965.0
-    alu_peak = SMS * FP32_LANES_PER_SM * mhz * 1e6 / 1e12
-    ach = prefill_instr(cfg, T) / (k_us * 1e-6) / 1e12
     gbs = prefill_bytes(cfg, T) / (k_us * 1e-6) / 1e9
-    return {"prompt_tokens": T, "handoff_us": round(pf_us[T], 2), "sketch_only_us": round(pf_us[0], 2),
-            "kernel_us": round(k_us, 2), "prompt_tok_s": round(cfg.B * T / (pf_us[T] * 1e-6), 1),
-            "roofline": {"kernel": "sketchssm_prefill", "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
-                         "unit": "GB/s", "frac": round(gbs / peak, 4), "peak_source": peak_src,
-                         "algorithmic_bytes_per_launch": prefill_bytes(cfg, T),
-                         "traffic": (lambda tr: None if tr is None else tr["dram_bytes_per_launch_full_size"])(
-                             kernel_traffic("sketchssm_prefill", cfg.name))},
-            "fp32_pipe": {"achieved": round(ach, 2), "peak": round(alu_peak, 2), "unit": "T FP32 lane-instr/s",
-                          "frac": round(ach / alu_peak, 4), "algorithmic_instr_per_launch": prefill_instr(cfg, T)}}
+    rep = {"prompt_tokens": T, "handoff_us": round(pf_us[T], 2), "sketch_only_us": round(pf_us[0], 2),
+           "kernel_us": round(k_us, 2), "prompt_tok_s": round(cfg.B * T / (pf_us[T] * 1e-6), 1),
+           "roofline": {"kernel": "sketchssm_prefill", "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                        "unit": "GB/s", "frac": round(gbs / peak, 4), "peak_source": peak_src,
+                        "algorithmic_bytes_per_launch": prefill_bytes(cfg, T),
+                        "traffic": (lambda tr: None if tr is None else tr["dram_bytes_per_launch_full_size"])(
+                            kernel_traffic("sketchssm_prefill", cfg.name))}}
+    if prefill_tensor_path(cfg, T):
+        fl = prefill_flops(cfg, T)
+        tp, tsrc = tf32_peak()
+        rep["tensor"] = {"achieved": round(fl["algorithmic"] / (k_us * 1e-6) / 1e12, 2),
+                         "issued": round(fl["issued"] / (k_us * 1e-6) / 1e12, 2), "peak": round(tp, 1),
+                         "unit": "TFLOP/s", "frac_issued": round(fl["issued"] / (k_us * 1e-6) / 1e12 / tp, 4),
+                         "peak_source": tsrc, "flops_per_launch": fl}
+    else:
+        mhz = clocks.get("sm_max_mhz") or 1965.0
+        alu_peak = SMS * FP32_LANES_PER_SM * mhz * 1e6 / 1e12
+        ach = prefill_instr(cfg, T) / (k_us * 1e-6) / 1e12
+        rep["fp32_pipe"] = {"achieved": round(ach, 2), "peak": round(alu_peak, 2), "unit": "T FP32 lane-instr/s",
+                            "frac": round(ach / alu_peak, 4), "algorithmic_instr_per_launch": prefill_instr(cfg, T)}
+    return rep
 
 
 def run_reference(args, cfg) -> None:

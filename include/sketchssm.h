@@ -141,13 +141,15 @@ sketchssm_status sketchssm_plan_query(const sketchssm_plan *plan, int64_t *r_tot
 
 /*
  * Synchronise `stream`, then report what the kernels recorded on the plan since the
- * last check, and clear it: SKETCHSSM_ERR_TIMEOUT if a decode or flush CTA waited
- * longer than the plan's wait limit (sketchssm_plan_set_wait_limit; default about a
- * second) for its own bulk copies; SKETCHSSM_OK otherwise.  Such a CTA records the
- * timeout and keeps waiting, up to the default limit more, for the same copies, so
- * the outputs are complete unless that second wait also ran out (then the CTA gives
- * up and its outputs are incomplete).  No kernel waits on anything but its own copies,
- * so a timeout at the default limit means a fault of the copy engine, not a deadlock.
+ * last check, and clear it: SKETCHSSM_ERR_TIMEOUT if a decode, flush, standard-step or
+ * prefill CTA waited longer than the plan's wait limit (sketchssm_plan_set_wait_limit;
+ * default about a second) for its own bulk copies (the Mamba-2 prefill: for its own
+ * tensor-core products); SKETCHSSM_OK otherwise.  Such a CTA records the timeout and
+ * keeps waiting, up to the default limit more, for the same operations, so the outputs
+ * are complete unless that second wait also ran out (then the CTA gives up and its
+ * outputs are incomplete).  No kernel waits on anything but its own operations, so a
+ * timeout at the default limit means a fault of the copy engine or the tensor core, not
+ * a deadlock.
  */
 sketchssm_status sketchssm_plan_check(const sketchssm_plan *plan, sketchssm_stream stream);
 

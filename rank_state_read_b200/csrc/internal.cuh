@@ -20,6 +20,7 @@ constexpr int SK_STATUS_DECODE_TIMEOUT = 1;
 constexpr int SK_STATUS_FLUSH_TIMEOUT = 2;
 constexpr int SK_STATUS_STEP_TIMEOUT = 4;
 constexpr int SK_STATUS_BAD_ROW = 8;  // a per-row position or token count out of range
+constexpr int SK_STATUS_PREFILL_TIMEOUT = 16;
 
 // default bound of a kernel's wait on its own bulk copies (clock cycles, ~1 s)
 constexpr long long DEFAULT_WAIT_CYCLES = 2000000000LL;
@@ -106,8 +107,13 @@ struct PrefillArgs {
     int VS;
     const float *k, *v, *a, *beta;
     float *S;
+    int *status;           // plan status word (timeouts of the tensor-core waits)
+    long long wait_limit;  // clock cycles of a bounded wait
 };
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream);
+// Mamba-2 prompts of at most 64 tokens with V a multiple of 16 up to 128: the tcgen05 kernel
+bool prefill_tcgen05_fits(const PrefillArgs &a);
+cudaError_t launch_prefill_tcgen05(const PrefillArgs &a, cudaStream_t stream);
 
 int flush_slab(int V);
 size_t flush_smem_bytes(int kind, int V, int W, int rcap);

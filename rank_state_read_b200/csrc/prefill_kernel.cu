@@ -407,6 +407,7 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t stream)
     if (a.B == 0 || a.T == 0) return cudaSuccess;
     switch (a.kind) {
     case SKETCHSSM_MAMBA2: {
+        if (prefill_tcgen05_fits(a)) return launch_prefill_tcgen05(a, stream);
         const size_t smem = tc_carve(a.VS).total;
         cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

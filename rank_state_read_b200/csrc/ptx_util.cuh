@@ -1,5 +1,5 @@
-// Inline-PTX helpers for the Blackwell data-movement paths: mbarriers and the bulk
-// (TMA, non-tensor) global -> shared copy, plus Ampere-style cp.async.
+// Inline-PTX helpers for the Blackwell paths: mbarriers, the bulk (TMA, non-tensor)
+// global -> shared copy, Ampere-style cp.async, and the tcgen05 tensor-memory MMA.
 //
 // Only the plain CTA-local forms are used: no cluster multicast anywhere.
 #pragma once
@@ -132,6 +132,99 @@ __device__ __forceinline__ void pdl_launch_dependents()
 __device__ __forceinline__ void pdl_wait_primary()
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- tcgen05 (tensor memory)
+// The 5th-generation tensor-core path: operands in shared memory described by matrix
+// descriptors, the fp32 accumulator in tensor memory (128 lanes x up to 512 32-bit
+// columns per SM), the MMA issued by one thread and its completion signalled on an
+// mbarrier.  Only the single-CTA (cta_group::1) forms are used.
+
+// allocate `cols` tensor-memory columns (a power of two, at least 32) for this CTA; one
+// whole warp executes it and the column address lands in *dst (shared memory)
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t cols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)), "r"(cols)
+                 : "memory");
+}
+
+// let other CTAs on this SM allocate (after this CTA's single allocation)
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+// free the allocation (the warp that allocated, before the CTA exits)
+__device__ __forceinline__ void tmem_dealloc(uint32_t addr, uint32_t cols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(addr), "r"(cols) : "memory");
+}
+
+// order tensor-core operations across a thread barrier (before it / after it)
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// make this thread's ordinary shared-memory writes visible to the async proxy (the
+// tensor core reads its operands through it)
+__device__ __forceinline__ void fence_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor without swizzling: start address, the byte distance
+// between adjacent 8 x 16-byte core matrices along the K dimension (`lbo`) and along
+// the M / N dimension (`sbo`), all in 16-byte units, and the descriptor version 1 of
+// this architecture in bits 46-47.
+__device__ __forceinline__ uint64_t umma_sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor of a dense tf32 x tf32 -> fp32 MMA with both operands K-major:
+// accumulator format fp32 (bits 4-5 = 1), A and B format tf32 (bits 7-9, 10-12 = 2),
+// N / 8 in bits 17-22, M / 16 in bits 24-28.
+__host__ __device__ constexpr uint32_t umma_idesc_tf32(int M, int N)
+{
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (accumulate ? D : 0) + A B over one K step (8 tf32 values), issued by one thread
+__device__ __forceinline__ void umma_tf32(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// one arrival on `bar` once every MMA this thread has issued so far has completed
+__device__ __forceinline__ void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// 16 consecutive 32-bit columns of the warp's 32 tensor-memory lanes (lane i of the warp
+// reads lane (addr >> 16) + i), waited for before returning
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, float (&x)[16])
+{
+    uint32_t r[16];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(addr)
+                 : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 16; ++j) x[j] = __uint_as_float(r[j]);
 }
 
 }  // namespace sk

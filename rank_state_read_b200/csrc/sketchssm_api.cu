@@ -388,6 +388,8 @@ sketchssm_status sketchssm_plan_check(const sketchssm_plan *p, sketchssm_stream 
         return fail(SKETCHSSM_ERR_TIMEOUT, "a standard-step CTA waited past the plan's limit for its bulk copies");
     if (flags & sk::SK_STATUS_FLUSH_TIMEOUT)
         return fail(SKETCHSSM_ERR_TIMEOUT, "a flush CTA waited past the plan's limit for its bulk copies");
+    if (flags & sk::SK_STATUS_PREFILL_TIMEOUT)
+        return fail(SKETCHSSM_ERR_TIMEOUT, "a prefill CTA waited past the plan's limit for its tensor-core products");
     return SKETCHSSM_OK;
 }
 
@@ -679,6 +681,8 @@ extern "C" sketchssm_status sketchssm_prefill(const sketchssm_plan *p, int32_t T
         A.a = a;
         A.beta = beta;
         A.S = S;
+        A.status = p->d_status;
+        A.wait_limit = p->wait_limit;
         cudaError_t e = sk::launch_prefill(A, (cudaStream_t)stream);
         if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
     }

@@ -52,6 +52,21 @@ def test_prefill_instruction_counts():
         assert bench.prefill_instr(cfg, 64) == per * cfg.B * cfg.H * cfg.K * cfg.V * 64
 
 
+def test_prefill_tensor_work_of_the_mamba2_layer():
+    """The 64-token Mamba-2 prompt runs on the tensor cores: 2 K V T FLOPs per head of
+    contraction; the kernel issues three tf32 products of 128 x 128 x 64 per head."""
+    cfg = synth.config(1)
+    assert bench.prefill_tensor_path(cfg, 64) and not bench.prefill_tensor_path(cfg, 65)
+    assert not bench.prefill_tensor_path(synth.config(3), 64)
+    assert bench.prefill_tensor_path(cfg.replace(V=128), 64)
+    assert not bench.prefill_tensor_path(cfg.replace(V=144), 64)
+    fl = bench.prefill_flops(cfg, 64)
+    heads = 256 * 128
+    assert fl["algorithmic"] == heads * 2 * 128 * 80 * 64
+    assert fl["issued"] == heads * 3 * 2 * 128 * 128 * 64
+    assert bench.prefill_flops(cfg, 61)["issued"] == fl["issued"]  # the prompt padded to 8
+
+
 def test_prefill_bytes_of_the_mamba2_layer():
     """The prefill reads and writes the state once and reads every prompt token:
     2 x 256 x 128 x 128 x 80 x 4 bytes + 64 tokens x 256 rows x (8 x 128 + 128 x 80 + 128) x 4."""

@@ -1,7 +1,8 @@
 """The prefill handoff (sketchssm_prefill) against the fp64 oracle (``oracle.prefill``
 followed by the n = 0 flush): the state and the sketch after prompts that span several
-token chunks and end in a ragged tail, prompts of 0 and exactly one or two chunks, and
-the decode steps that follow the handoff from pos = 0.
+token chunks and end in a ragged tail, prompts of 0 and exactly one or two chunks,
+Mamba-2 prompts on both sides of the tensor-memory kernel's limits (64 tokens, value
+widths up to 128), and the decode steps that follow the handoff from pos = 0.
 
 Bar: max |gpu - oracle| / max |oracle| <= 1e-4 for S, Y and every y.
 """
@@ -72,6 +73,21 @@ def test_prefill_small(cid, B, T):
 def test_prefill_edge_lengths(cid, T):
     """No token (Y only), one token, exactly one and two chunks."""
     prefill_parity(synth.config(cid).replace(B=2), T)
+
+
+@pytest.mark.parametrize("T", [7, 63, 64, 65, 100])
+def test_prefill_mamba2_lengths(T):
+    """Mamba-2 prompts around the tensor-memory kernel's 64-token limit (a ragged last
+    K step, exactly 64, and longer prompts on the chunked kernel)."""
+    prefill_parity(synth.config(1).replace(B=3), T)
+
+
+@pytest.mark.parametrize("V", [16, 48, 112, 128, 160])
+def test_prefill_mamba2_value_dims(V):
+    """Mamba-2 value widths up to 128 on the tensor-memory kernel (whose 128-row value
+    operand reads past the last value row), V = 160 on the chunked one."""
+    cfg = synth.config(1).replace(B=2, V=V)
+    prefill_parity(cfg, 37)
 
 
 @pytest.mark.parametrize("V", [16, 48, 256])

@@ -1,4 +1,4 @@
-"""The bounded waits of the decode and flush kernels, made to run out on purpose.
+"""The bounded waits of the decode, flush and prefill kernels, made to run out on purpose.
 
 With the plan's wait limit at a few clock cycles, the CTAs' waits for their own bulk
 copies run past it: the kernels record a timeout, which sketchssm_plan_check reports
@@ -67,6 +67,30 @@ def test_short_wait_limit_is_reported_and_outputs_complete(cid):
     x = synth.device_step_inputs(cfg, 900, "cuda")
     short.decode(0, x["q"], x["k"], x["v"], x["a"], x["beta"])
     short.plan.check()
+    ref.close()
+    short.close()
+
+
+def test_short_wait_limit_in_the_tensor_core_prefill():
+    """The Mamba-2 prefill waits for its own tensor-core products: with a one-cycle limit
+    the waits overrun, the timeout is reported, and the state and sketch equal those of
+    a run at the default limit."""
+    import torch
+    import rank_state_read_b200 as rs
+    cfg = synth.config(1).replace(B=4)
+    rank = synth.layer_rank_table(cfg)
+    omega, S0 = synth.basis(cfg), synth.init_state(cfg, range(cfg.B))
+    ref, short = _layer(cfg, rank, omega, S0), _layer(cfg, rank, omega, S0)
+    p = {k: (None if v is None else torch.from_numpy(v).cuda()) for k, v in synth.prompt_inputs(cfg, 40, range(cfg.B)).items()}
+    ref.prefill(p["k"], p["v"], p["a"], p["beta"])
+    ref.plan.check()
+    short.plan.set_wait_limit(1)
+    short.prefill(p["k"], p["v"], p["a"], p["beta"])
+    with pytest.raises(rs.SketchSSMError) as err:
+        short.plan.check()
+    assert err.value.status == 5  # SKETCHSSM_ERR_TIMEOUT
+    torch.cuda.synchronize()
+    assert torch.equal(short.S, ref.S) and torch.equal(short.Y, ref.Y)
     ref.close()
     short.close()
 
