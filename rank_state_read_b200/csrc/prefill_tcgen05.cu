@@ -7,14 +7,19 @@
 //
 //     S_T = G S_0 + sum_t w_t k_t v_t^T,   w_t = prod_{t<j<T} a_j,   G = prod_{j<T} a_j,
 //
-// i.e. D[m][n] = sum_t K[m][t] B[t][n] with K[m][t] = k_t[m] and B[t][n] = w_t v_t[n].
+// taken transposed, D^T[n][m] = sum_t (w_t v_t[n]) k_t[m], so that tensor-memory lane n
+// holds value column n of the new state.
 //
-// One CTA per (batch row, q/k head) walks that q/k head's heads.  The prompt's keys
-// (shared by the heads) are staged once as the A operand; each head's weighted values
-// are the B operand; one thread issues the MMAs (M = 128 state rows, N = V, K = 8
-// tokens a step) into one of two tensor-memory accumulators, so that the MMAs of head j
-// run while the epilogue of head j - 1 (thread m: tensor-memory lane m = state row m,
-// plus G S_0 row m, written back) and the loads for head j + 1 proceed.
+// One CTA of 128 threads per (batch row, q/k head) walks that q/k head's heads, two CTAs
+// per SM.  The prompt's keys (shared by the heads) are staged once as the B operand
+// (N = 128 state rows); each head's weighted values w_t v_t[n] are the A operand (M = 128
+// rows: rows n >= V read whatever follows them and land in lanes nobody reads); one
+// thread of the last warp issues the MMAs (K = 8 tokens a step) into one of two
+// tensor-memory accumulators.  So the MMAs of head j run while the epilogue of head
+// j - 1 proceeds: thread n (lane n) adds G S_0[m][n] to D^T[n][m], 16 state rows m at a
+// time, and its warp writes each state row as 128 contiguous bytes.  Meanwhile the
+// loads for head j + 1 (its values) and head j (its S_0 column) are in flight into
+// registers.
 //
 // Precision: every operand x is split into hi = x with its 13 low mantissa bits cleared
 // (exact in tf32) and lo = x - hi (exact in fp32), and D accumulates hi*hi + hi*lo +
@@ -32,7 +37,7 @@
 namespace sk {
 namespace {
 
-constexpr int PU_THREADS = 128;  // one thread per state row = tensor-memory lane
+constexpr int PU_THREADS = 128;  // one thread per tensor-memory lane (value column)
 constexpr int PU_TMAX = 64;      // prompt tokens staged at once (longer prompts take the other kernel)
 
 __host__ __device__ constexpr int pu_round8(int x) { return (x + 7) & ~7; }

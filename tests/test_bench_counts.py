@@ -67,6 +67,22 @@ def test_prefill_tensor_work_of_the_mamba2_layer():
     assert bench.prefill_flops(cfg, 61)["issued"] == fl["issued"]  # the prompt padded to 8
 
 
+def test_prefill_report_carries_the_pipe_of_its_kernel():
+    """The prefill line reports the tensor pipe for the tcgen05 (Mamba-2) kernel and the
+    FP32 pipe for the others, and its HBM fraction is the algorithmic bytes over the
+    kernel time (the handoff minus the sketch-only call)."""
+    pf_us = {64: 1200.0, 0: 350.0}
+    clocks = {"sm_max_mhz": 1965.0}
+    m2 = bench.prefill_report(synth.config(1), pf_us, clocks, 6541.5, "measured")
+    assert "tensor" in m2 and "fp32_pipe" not in m2
+    assert m2["kernel_us"] == 850.0
+    gbs = bench.prefill_bytes(synth.config(1), 64) / 850e-6 / 1e9
+    assert abs(m2["roofline"]["frac"] - gbs / 6541.5) < 1e-4
+    assert m2["tensor"]["flops_per_launch"] == bench.prefill_flops(synth.config(1), 64)
+    gdn = bench.prefill_report(synth.config(3), pf_us, clocks, 6541.5, "measured")
+    assert "fp32_pipe" in gdn and "tensor" not in gdn
+
+
 def test_prefill_bytes_of_the_mamba2_layer():
     """The prefill reads and writes the state once and reads every prompt token:
     2 x 256 x 128 x 128 x 80 x 4 bytes + 64 tokens x 256 rows x (8 x 128 + 128 x 80 + 128) x 4."""
