@@ -94,7 +94,7 @@ def test_prefill_bytes_of_the_mamba2_layer():
 
 def test_state_traffic_ratio_of_the_shapes():
     """The state-only bytes per token of the standard step over those of the sketch path
-    (SURVEY's reconstruction of the pages' figure: 10.4x at rank 8, W = 16, K = 128,
+    (the analytic reconstruction of the pages' figure: 10.4x at rank 8, W = 16, K = 128,
     V = 80, no dense head)."""
     cfg = synth.config(1).replace(n_dense=0)
     rank = np.full(cfg.H, 8, np.int32)
