@@ -570,3 +570,34 @@ def test_sketch_read_is_the_exact_read_of_the_projected_state(kind):
         ys = sk.decode(t, inp)
         ye = ex.decode(t, inp, dense_all=True)
         assert rel(ys, ye) < 1e-12, t
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn", "kda"])
+@pytest.mark.parametrize("T", [3, 9])
+def test_prefill_equals_the_buffered_update_path(kind, T):
+    """The prompt path and the decode path update the state by the same recurrence: a
+    prompt applied by prefill leaves the same state and sketch as its tokens appended one
+    by one (decode, any query) with a flush after every W of them and one for the rest.
+    Two separate routines of the oracle, so a mistake in either shows."""
+    cfg = tiny_cfg(kind, Hqk=2 if kind == "mamba2" else None)
+    rank = np.array([1, DENSE, 2, 3], np.int32)
+    rows = list(range(cfg.B))
+    omega = synth.basis_fp64(cfg)
+    S0 = synth.init_state(cfg, rows)
+    mk = lambda: oracle.OracleLayer(cfg.kind, H=cfg.H, Hqk=cfg.Hqk, K=cfg.K, V=cfg.V, W=cfg.W,
+                                    G=cfg.G, rank=rank, omega=omega, S0=S0)
+    pre, dec = mk(), mk()
+    p = synth.prompt_inputs(cfg, T, rows)
+    pre.prefill(p)
+    pos = 0
+    for t in range(T):
+        tok = {"q": np.zeros((cfg.B, cfg.Hqk, cfg.K), np.float32), "k": p["k"][:, t], "v": p["v"][:, t],
+               "a": p["a"][:, t], "beta": None if p["beta"] is None else p["beta"][:, t]}
+        dec.decode(pos, tok)
+        pos += 1
+        if pos == cfg.W:
+            dec.flush(pos)
+            pos = 0
+    dec.flush(pos)
+    assert rel(dec.S, pre.S) < 1e-12
+    assert rel(dec.Y, pre.Y) < 1e-12
