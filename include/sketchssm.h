@@ -311,6 +311,9 @@ sketchssm_status sketchssm_step(const sketchssm_plan *plan, const float *q, cons
  *    beta [B][T][H] (NULL for Mamba-2).  k, v, a may be NULL when T = 0.
  *  - S [B][H][K][V] is read and written once whatever T; omega and Y as for
  *    sketchssm_flush.
+ *  - Mamba-2 prompts of at most 64 tokens with V <= 128 run on the tensor cores
+ *    (tcgen05, fp32 accuracy by a three-product tf32 split); other prompts and kinds
+ *    apply the tokens in 16-token chunks.
  *  - T < 0 returns SKETCHSSM_ERR_INVALID_ARG; nothing is launched on an error.
  */
 sketchssm_status sketchssm_prefill(const sketchssm_plan *plan, int32_t T, const float *k, const float *v,

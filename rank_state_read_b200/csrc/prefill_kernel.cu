@@ -11,6 +11,8 @@
 // buffered with cp.async: chunk c + 1 is in flight while the CTA applies chunk c.  No
 // thread waits on another CTA or on a flag: the only waits are cp.async groups and CTA
 // barriers.
+//   Mamba-2 prompts of at most 64 tokens with V a multiple of 16 up to 128 go to the
+//   tcgen05 kernel (prefill_tcgen05.cu); the others:
 //   Mamba-2 (prefill_tc_kernel): a chunk of n tokens is one contraction,
 //     S <- P S + K^T (w o V), w_i = product of the later decays in the chunk, P of all,
 //     on the tensor cores (mma.sync m16n8k8, tf32 operands split hi + lo, three
